@@ -1,0 +1,27 @@
+"""Compile the CPU oracle (test infrastructure only) into oracle/_liboracle.so.
+
+Usage: python -m oracle.build   (also run by __graft_entry__.build()).
+"""
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "sgmv_oracle.c")
+LIB = os.path.join(HERE, "_liboracle.so")
+
+
+def build(force: bool = False, out: str = LIB, defines=()) -> str:
+    """Compile the oracle.  `defines` (e.g. ["ORC_MUTANT=3"]) is for the mutation test only."""
+    if not force and not defines and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(SRC):
+        return out
+    # -ffp-contract=off: the oracle's products and sums are separate fp64
+    # operations, each rounded, exactly as written in the source.
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
+           "-std=c11", "-Wall", *["-D" + d for d in defines], "-o", out + ".tmp", SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    return out
+
+
+if __name__ == "__main__":
+    print(build(force=True))

@@ -1,0 +1,554 @@
+"""Benchmark of SGMV expand-slice on B200.
+
+One step = the whole hot path over one batch: the three expand-slice calls of a
+Llama-7B fused-QKV prefill batch (16 sequences with lengths uniform in
+[64, 1024], rank 16, 32 adapters with 10% of sequences at -1, bf16, slices of
+4096 at offsets 0/4096/8192 of a T x 12288 output, add_inputs=True).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--variant auto|simt|tc]
+
+Timing: inputs are resident in HBM; W untimed warm-up steps; then K steps as
+CUDA-graph replays (each graph holds up to 100 steps, with an event recorded
+on the launching stream before and after every kernel), bracketed by a barrier
+and a device synchronise on both sides; max over ranks.  The output (215 MB
+for the default workload) is larger than L2 and every step streams all of it,
+so no flush is needed between steps.  `value` is algorithmic HBM bytes of all
+ranks / time; `e2e` repeats the measurement through the same C-ABI calls with
+the inputs in pinned host memory, copying them in and the output back every
+step.  `--impl reference` times the CPU oracle on host cores instead (rank 0).
+"""
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sgmv_inputs as gen  # noqa: E402
+
+METRIC = "sgmv_expand_slice achieved HBM GB/s (% of B200 roofline) and tokens/s per call"
+FALLBACK_HBM_GBS = 6650.0
+STEPS_PER_GRAPH = 100
+
+WORKLOAD_TEXT = {
+    "qkv_prefill": "Llama-7B fused-QKV prefill: 16 seqs U[64,1024], rank 16, 32 adapters (10% idx -1), "
+                   "bf16, 3 slices of 4096 into T x 12288, add_inputs",
+    "mlp_mixed": "MLP gate/up: 64 seqs Geom(mean 256)<=2048, rank 64, fp32 x vs bf16 4-D weights "
+                 "(128 adapters), bf16 out T x 22016, 2 slices of 11008, add_inputs",
+    "long_single": "single-tenant long prefill: 1 x 32768 tokens, rank 8, fp16, 4096 slice, overwrite",
+    "decode_mix": "decode-like mix: 256 seqs Zipf(1.2) in [1,64], rank 32, 256 distinct adapters "
+                  "(10% -1), bf16, slice 5120 at 5120 of T x 15360, add_inputs",
+    "tiny": "tiny: 4 seqs [4,6,3,7], rank 16, fp16, slice 128 at 128, overwrite",
+}
+
+DT_SIZE = {"f16": 2, "bf16": 2, "f32": 4}
+
+
+# ---------------------------------------------------------------- accounting
+
+def call_accounting(p: gen.Problem, call: int):
+    """Algorithmic bytes and flops of one expand-slice call, from the metadata."""
+    c = p.calls[call]
+    A, N, K = c.w.shape[0], c.slice_size, p.rank
+    ok = (p.lora_idx >= 0) & (p.lora_idx < A) & (p.seq_len > 0) & (p.seq_start >= 0)
+    rows = int(p.seq_len[ok].sum())
+    adapters = len(np.unique(p.lora_idx[ok]))
+    meta = 3 * p.batches * (8 if p.meta_dt == "int64" else 4)
+    sx, sw, so = DT_SIZE[p.x_dt], DT_SIZE[p.w_dt], DT_SIZE[p.out_dt]
+    byts = rows * (K * sx + N * so * (2 if p.add_inputs else 1)) + adapters * N * K * sw + meta
+    flops = 2 * N * K * rows
+    return byts, flops, rows
+
+
+def step_accounting(p):
+    b = f = r = 0
+    for c in range(len(p.calls)):
+        bb, ff, rr = call_accounting(p, c)
+        b, f, r = b + bb, f + ff, r + rr
+    return b, f, r
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "segmented_gather_gemm_expand_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, variant):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        e = d[workload][variant]
+        if e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sgmv_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.bus_id and self.bus_id not in parts[1].lower():
+                continue
+            rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][3]) if rows[0][3].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- runtime helpers
+
+def cudart():
+    import torch
+    lib_dir = os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib")
+    for cand in [os.path.join(lib_dir, "libcudart.so.12"), "libcudart.so.12", "libcudart.so"]:
+        try:
+            lib = ctypes.CDLL(cand)
+            break
+        except OSError:
+            continue
+    lib.cudaEventCreate.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+    lib.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+    lib.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
+    lib.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+    return lib
+
+
+class Events:
+    """Raw CUDA events recorded as graph nodes (cudaEventRecordExternal)."""
+
+    def __init__(self, rt, n):
+        self.rt = rt
+        self.ev = []
+        for _ in range(n):
+            h = ctypes.c_void_p()
+            assert rt.cudaEventCreate(ctypes.byref(h)) == 0
+            self.ev.append(h)
+
+    def record(self, i, stream_handle):
+        assert self.rt.cudaEventRecordWithFlags(self.ev[i], ctypes.c_void_p(stream_handle), 1) == 0
+
+    def elapsed_ms(self, i, j):
+        out = ctypes.c_float()
+        assert self.rt.cudaEventElapsedTime(ctypes.byref(out), self.ev[i], self.ev[j]) == 0
+        return out.value
+
+    def destroy(self):
+        for h in self.ev:
+            self.rt.cudaEventDestroy(h)
+
+
+def make_calls(p, dev_tensors, sg_abi, stream_handle_fn):
+    """Pre-marshalled C-ABI argument tuples, one per slice call."""
+    import segmented_gather_gemm_expand_b200 as sg
+    x, ws, y, meta = dev_tensors
+    descs = []
+    for c, call in enumerate(p.calls):
+        d = [sg._desc(t) for t in (x, ws[c], y, *meta)]
+        descs.append((d, call.slice_offset, call.slice_size))
+    lib = sg._lib
+
+    def run(c, stream):
+        d, off, size = descs[c]
+        rc = lib.sgmv_expand_slice(*[ctypes.byref(t) for t in d], p.batches, p.max_seq_len, off, size,
+                                   int(p.add_inputs), ctypes.c_void_p(stream))
+        if rc != 0:
+            raise sg.SgmvError(rc, "sgmv_expand_slice")
+    return run, descs
+
+
+# ---------------------------------------------------------------- our arm
+
+def bench_ours(args, rank, world, device):
+    import torch
+    import segmented_gather_gemm_expand_b200 as sg
+    from segmented_gather_gemm_expand_b200 import _abi
+
+    torch.cuda.set_device(device)
+    variants = {"auto": sg.VARIANT_AUTO, "simt": sg.VARIANT_SIMT, "tc": sg.VARIANT_TC}
+    sg.set_variant(variants[args.variant])
+    p = gen.WORKLOADS[args.workload](seed=args.seed + rank)
+    tdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+    def host_tensor(a, dt):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if dt != "f32" else np.ascontiguousarray(a))
+        return t.view(tdt[dt]) if dt != "f32" else t
+
+    hx = host_tensor(p.x, p.x_dt)
+    hws = [host_tensor(c.w, p.w_dt) for c in p.calls]
+    hy = host_tensor(p.y0, p.out_dt)
+    hmeta = [torch.from_numpy(a.astype(np.int64)) for a in (p.seq_start, p.seq_len, p.lora_idx)]
+    x = hx.to(device)
+    ws = [w.to(device) for w in hws]
+    y = hy.to(device)
+    meta = [m.to(device) for m in hmeta]
+    run, _ = make_calls(p, (x, ws, y, meta), _abi, None)
+    ncalls = len(p.calls)
+    v_used = sg.plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, p.calls[0].slice_offset,
+                     p.calls[0].slice_size, p.add_inputs)
+    variant_name = {1: "simt", 2: "tc"}.get(v_used, str(v_used))
+
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for c in range(ncalls):
+                run(c, stream.cuda_stream)
+    torch.cuda.synchronize()
+
+    # Capture the timed steps as graphs with an event around every launch.
+    rt = cudart()
+    K = args.steps
+    graphs, evsets = [], []
+    remaining = K
+    while remaining > 0:
+        s = min(STEPS_PER_GRAPH, remaining)
+        ev = Events(rt, 2 * s * ncalls)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            cs = torch.cuda.current_stream().cuda_stream
+            i = 0
+            for _ in range(s):
+                for c in range(ncalls):
+                    ev.record(i, cs)
+                    run(c, cs)
+                    ev.record(i + 1, cs)
+                    i += 2
+        graphs.append(g)
+        evsets.append(ev)
+        remaining -= s
+    # one untimed replay of every graph (first-launch costs)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+
+    bus = None
+    try:
+        pr = torch.cuda.get_device_properties(device)
+        bus = f"{int(pr.pci_bus_id):02x}:{int(pr.pci_device_id):02x}."
+    except Exception:
+        pass
+    sampler = ClockSampler(bus)
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for g in graphs:
+            g.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = []
+    for ev in evsets:
+        for i in range(0, len(ev.ev), 2):
+            launch_ms.append(ev.elapsed_ms(i, i + 1))
+    for ev in evsets:
+        ev.destroy()
+    del graphs
+    assert sg.device_error(device) == 0, "a kernel reported a device-side error"
+
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+
+    step_bytes, step_flops, step_rows = step_accounting(p)
+    call_bytes, _, _ = call_accounting(p, 0)
+    if world > 1:
+        tot = torch.tensor([step_bytes, step_flops, p.total_tokens], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(tot)
+        all_bytes, all_flops, all_tokens = [float(v) for v in tot.tolist()]
+    else:
+        all_bytes, all_flops, all_tokens = float(step_bytes), float(step_flops), float(p.total_tokens)
+    ms_per_step = total_ms / K
+    value = all_bytes * K / (total_ms * 1e-3) / 1e9
+    avg_launch_ms = float(np.mean(launch_ms))
+    achieved = call_bytes / (avg_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+
+    # ---- end to end: pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        phx, phy = hx.pin_memory(), hy.pin_memory()
+        phws = [w.pin_memory() for w in hws]
+        phmeta = [m.pin_memory() for m in hmeta]
+        out_host = torch.empty_like(phy).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in [phx, phy, *phws, *phmeta])
+        d2h = out_host.numel() * out_host.element_size()
+        E = args.e2e_steps
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(E):
+                x.copy_(phx, non_blocking=True)
+                y.copy_(phy, non_blocking=True)
+                for w, pw in zip(ws, phws):
+                    w.copy_(pw, non_blocking=True)
+                for m, pm in zip(meta, phmeta):
+                    m.copy_(pm, non_blocking=True)
+                for c in range(ncalls):
+                    run(c, stream.cuda_stream)
+                out_host.copy_(y, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": all_bytes * E / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms / E, "steps": E}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(p, budget_s=args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": p.w_dt, "accumulate": "f32",
+        "data": "synthetic (seeded numpy; inputs resident in HBM)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
+                   "batches": p.batches, "tokens_per_rank": p.total_tokens,
+                   "active_tokens_per_rank": step_rows // max(ncalls, 1), "rank": p.rank,
+                   "slices": ncalls, "slice_size": p.calls[0].slice_size,
+                   "adapters": int(p.calls[0].w.shape[0]), "add_inputs": bool(p.add_inputs),
+                   "x_dtype": p.x_dt, "w_dtype": p.w_dt, "out_dtype": p.out_dt,
+                   "parallelism": f"replicas x{world} (independent batches, no collective)",
+                   "l2": "no flush: every step streams the whole output, larger than L2",
+                   "variant": variant_name, "seed": args.seed,
+                   "timing": f"CUDA graphs of <= {STEPS_PER_GRAPH} steps, events around every launch"},
+        "tokens_per_s": all_tokens * ncalls / (total_ms * 1e-3) / ncalls,
+        "tokens_per_s_note": "tokens of one call / average call time (per call, all ranks)",
+        "tflops": all_flops * K / (total_ms * 1e-3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload, variant_name),
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6650 GB/s",
+                     "kernel": f"sgmv expand-slice ({variant_name})",
+                     "launch_ms_avg": avg_launch_ms, "bytes_per_launch": call_bytes,
+                     "launches_timed": len(launch_ms)},
+        "gpu_launches": K * ncalls,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "when": datetime.datetime.utcnow().isoformat() + "Z",
+    }
+    return line
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(p, rows_budget, rng):
+    """A compact problem made of the first rows of randomly chosen sequences of
+    the workload (about rows_budget active rows): the chosen rows of x and of
+    the output are copied out, and the segments renumbered onto them."""
+    A = p.calls[0].w.shape[0]
+    valid = [b for b in range(p.batches) if 0 <= p.lora_idx[b] < A and p.seq_len[b] > 0]
+    order = rng.permutation(valid)
+    rows, lens, idx = [], [], []
+    left = rows_budget
+    for b in order:
+        if left <= 0:
+            break
+        take = int(min(p.seq_len[b], left))
+        rows.append(np.arange(p.seq_start[b], p.seq_start[b] + take))
+        lens.append(take)
+        idx.append(p.lora_idx[b])
+        left -= take
+    rows = np.concatenate(rows)
+    lens = np.array(lens, np.int64)
+    return gen.Problem(p.name, np.ascontiguousarray(p.x[rows]), p.x_dt, p.w_dt,
+                       np.ascontiguousarray(p.y0[rows]), p.out_dt, gen.exclusive_cumsum(lens), lens,
+                       np.array(idx, np.int64), p.add_inputs, p.calls)
+
+
+def run_oracle_sample(sub, nthreads):
+    import oracle
+    out = sub.y0
+    t0 = time.perf_counter()
+    for c in range(len(sub.calls)):
+        out = oracle.run_problem(sub, out=out, call=c, nthreads=nthreads)
+    return time.perf_counter() - t0, sub
+
+
+def cpu_baseline(p, budget_s=15.0, nthreads=None):
+    import oracle
+    nthreads = nthreads or oracle.max_threads()
+    rng = np.random.default_rng(0)
+    # calibrate on a small sample, then size the measured one to the budget
+    dt, sub = run_oracle_sample(oracle_sample(p, 8, rng), nthreads)
+    rows_per_s = max(int(sub.seq_len.sum()), 1) / max(dt, 1e-6)
+    rows = int(max(8, min(rows_per_s * budget_s, p.seq_len.sum())))
+    dt, sub = run_oracle_sample(oracle_sample(p, rows, np.random.default_rng(1)), nthreads)
+    b, _, r = step_accounting(sub)
+    return {"value": b / dt / 1e9, "unit": "GB/s", "cores": int(nthreads), "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{int(sub.seq_len.sum())} active rows from {len(sub.seq_len)} sequences of the same "
+                      f"workload, all {len(p.calls)} slices (fp64 C triple loop, OpenMP over rows)"}
+
+
+def bench_reference(args, rank, world):
+    """The CPU oracle, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    p = gen.WORKLOADS[args.workload](seed=args.seed)
+    nthreads = oracle.max_threads()
+    # rows per step so that warm-up + steps take about args.cpu_seconds
+    dt, sub = run_oracle_sample(oracle_sample(p, 8, np.random.default_rng(0)), nthreads)
+    rows_per_s = max(int(sub.seq_len.sum()), 1) / max(dt, 1e-6)
+    per_step = int(max(1, min(rows_per_s * args.cpu_seconds / max(args.steps + args.warmup, 1),
+                              p.seq_len.sum())))
+    rng = np.random.default_rng(2)
+    for _ in range(args.warmup):
+        run_oracle_sample(oracle_sample(p, per_step, rng), nthreads)
+    tot_t = 0.0
+    tot_b = 0
+    rows = 0
+    for _ in range(args.steps):
+        dt, sub = run_oracle_sample(oracle_sample(p, per_step, rng), nthreads)
+        b, _, r = step_accounting(sub)
+        tot_t += dt
+        tot_b += b
+        rows += int(sub.seq_len.sum())
+    value = tot_b / tot_t / 1e9
+    sample_txt = (f"{per_step} active rows per step drawn from the {args.workload} workload, all "
+                  f"{len(p.calls)} slices; fp64 C triple loop with OpenMP over rows")
+    return {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_t / max(args.steps, 1) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "seed": args.seed},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                             "sample": sample_txt},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(gen.WORKLOADS), default="qkv_prefill")
+    ap.add_argument("--variant", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = bench_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    device = torch.device("cuda", local)
+    if world > 1:
+        torch.cuda.set_device(device)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line = bench_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

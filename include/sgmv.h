@@ -1,0 +1,179 @@
+/*
+ * libsgmv -- SGMV expand-slice for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Implementation: Predibase Lorax SGMV Expand Slice Kernel",
+ * sections Description, Signature, I/O Contract and Outputs): for every
+ * sequence b < batches with start s_b = seq_start[b], length L_b = seq_len[b]
+ * and adapter a = lora_idx[b], and every token m < L_b (row r = s_b + m),
+ *
+ *     out[r, off + n] = (add_inputs ? out[r, off + n] : 0) + sum_k x^[r, k] * B[a][n, k]
+ *
+ * for n in [0, slice_size), off = slice_offset.  x^ is x rounded to nearest-even
+ * in the weights' dtype ("mixed-precision type casting"); products are summed
+ * in fp32 and the sum (plus the old value when add_inputs) is rounded to
+ * nearest-even in out's dtype once.  Every other element of out keeps its bits:
+ * columns outside [off, off + slice_size), rows of segments whose adapter is -1,
+ * rows not covered by any segment.
+ *
+ * Conventions for every entry point:
+ *   - Memory: all tensor data pointers are DEVICE pointers on the current CUDA
+ *     device.  The caller owns every buffer; the library keeps no pointer after
+ *     a call returns and allocates no device memory.
+ *   - Streams: work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream).  Nothing synchronises the host, except where a function
+ *     says so.
+ *   - Errors: a negative status is returned BEFORE anything is enqueued, and
+ *     nothing is written, when an argument is invalid.  SGMV_ERR_CUDA /
+ *     SGMV_ERR_LAUNCH report a failing CUDA call (the launch may or may not
+ *     have been enqueued).  sgmv_status_string() names every code.
+ *   - Values inside device tensors (segment starts, lengths, adapter ids)
+ *     cannot be checked without a host synchronisation, so the kernels guard
+ *     them instead: a segment whose adapter id is outside [0, lora_num), whose
+ *     start is negative or whose length is not positive is skipped; rows at or
+ *     beyond the row count of `out` or of `inputs` are skipped.  No kernel
+ *     reads or writes outside the tensors it is given.  sgmv_validate_metadata()
+ *     reports such values without trapping.
+ *   - max_seq_len is accepted for signature parity with the page's wrapper,
+ *     where it sizes the launch grid; here the grid depends only on the SM
+ *     count and the work is expanded from the metadata on the device, so every
+ *     token m < L_b is processed even if max_seq_len is smaller.
+ */
+#ifndef SGMV_H
+#define SGMV_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SGMV_API __attribute__((visibility("default")))
+#else
+#define SGMV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types. */
+typedef enum {
+    SGMV_F16 = 0,   /* IEEE binary16 */
+    SGMV_BF16 = 1,  /* bfloat16 */
+    SGMV_F32 = 2,   /* IEEE binary32 */
+    SGMV_I32 = 3,   /* metadata only */
+    SGMV_I64 = 4    /* metadata only */
+} sgmv_dtype;
+
+/* A strided view of device memory.  shape[i] and stride[i] (in ELEMENTS, not
+ * bytes) are meaningful for i < ndim; the rest are ignored. */
+typedef struct {
+    void* data;
+    int32_t dtype;      /* sgmv_dtype */
+    int32_t ndim;       /* 1 .. 4 */
+    int64_t shape[4];
+    int64_t stride[4];
+} sgmv_tensor;
+
+/* Status codes. */
+enum {
+    SGMV_OK = 0,
+    SGMV_ERR_NULL_ARG = -1,          /* a descriptor or a non-empty tensor's data is NULL */
+    SGMV_ERR_DTYPE = -2,             /* a tensor's dtype is not allowed for its role */
+    SGMV_ERR_NDIM = -3,              /* wrong number of dimensions */
+    SGMV_ERR_RANK_MISMATCH = -4,     /* inputs.shape[1] != lora_b.shape[-1] */
+    SGMV_ERR_SLICE_SIZE = -5,        /* slice_size != lora_b.shape[-2] */
+    SGMV_ERR_LAYOUT_4D = -6,         /* 4-D lora_b whose dimension 1 is not 1 */
+    SGMV_ERR_OUT_NOT_CONTIGUOUS = -7,/* out is not contiguous row-major */
+    SGMV_ERR_SLICE_RANGE = -8,       /* slice_offset < 0 or slice_offset + slice_size > out.shape[1] */
+    SGMV_ERR_BATCHES = -9,           /* batches < 0, or a metadata tensor shorter than batches */
+    SGMV_ERR_SHAPE = -10,            /* a negative extent, or max_seq_len < 0 */
+    SGMV_ERR_STRIDE = -11,           /* a negative stride */
+    SGMV_ERR_TOO_LARGE = -12,        /* sizes beyond the library's index range */
+    SGMV_ERR_VARIANT = -13,          /* the forced kernel variant cannot run this call */
+    SGMV_ERR_CUDA = -20,             /* a CUDA runtime call failed */
+    SGMV_ERR_LAUNCH = -21            /* a kernel launch failed */
+};
+
+/* Kernel variants (for sgmv_set_variant / sgmv_plan). */
+enum {
+    SGMV_VARIANT_AUTO = 0,
+    SGMV_VARIANT_SIMT = 1,   /* generic CUDA-core kernel: any strides, rank, alignment */
+    SGMV_VARIANT_TC = 2      /* tcgen05 tensor-core kernel with TMA staging */
+};
+
+/*
+ * sgmv_expand_slice -- the operation above, in place on `out`.
+ *
+ *   inputs    (T_x, K)                    f16 | bf16 | f32, any non-negative strides
+ *   lora_b    (lora_num, N, K) or (lora_num, 1, N, K)   f16 | bf16, any strides;
+ *             N must equal slice_size; the 4-D form's unit dimension is dropped
+ *   out       (T_out, H)                  f16 | bf16 | f32, contiguous row-major
+ *   seq_start, seq_len, lora_idx  1-D, i32 | i64 (each independently), length
+ *             >= batches, any stride; lora_idx == -1 means "no LoRA"
+ *   batches, max_seq_len, slice_offset, slice_size, add_inputs: as in the page's
+ *             wrapper (sgmv_expand_slice's arguments of the same names).
+ *
+ * Returns SGMV_OK when the work was enqueued, or a negative status.  Calls with
+ * batches == 0, slice_size == 0 or T_out == 0 return SGMV_OK and enqueue nothing.
+ * Segments must not overlap (rows written by two segments are undefined).
+ */
+SGMV_API int sgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+                      const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                      const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
+                      int64_t slice_offset, int64_t slice_size, int add_inputs, void* stream);
+
+/*
+ * sgmv_plan -- validate exactly as sgmv_expand_slice does and report, in
+ * *variant, the kernel variant a call with these arguments would launch
+ * (SGMV_VARIANT_SIMT or SGMV_VARIANT_TC; 0 when nothing would launch).
+ * Launches nothing and touches no tensor data.  May query the current device's
+ * properties (once per device).
+ */
+SGMV_API int sgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+              const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+              int64_t batches, int64_t max_seq_len, int64_t slice_offset, int64_t slice_size,
+              int add_inputs, int* variant);
+
+/*
+ * sgmv_validate_metadata -- check the VALUES of the metadata on the device and
+ * write a bit mask to *d_status (a device int32; 0 = all well):
+ *   1   some lora_idx[b] is < -1 or >= lora_num
+ *   2   some seq_start[b] < 0 or seq_len[b] < 0
+ *   4   some segment (with a valid adapter) ends past total_rows
+ *   8   two segments with valid adapters overlap
+ *   16  starts of valid segments are not non-decreasing (overlap was then
+ *       checked pairwise, or not at all when batches > 8192 -- bit 32 set)
+ *   32  the pairwise overlap check was skipped
+ * Never traps.  Enqueued on `stream`; the caller reads *d_status after
+ * synchronising.  Same tensor rules as sgmv_expand_slice.
+ */
+SGMV_API int sgmv_validate_metadata(const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                           const sgmv_tensor* lora_idx, int64_t batches, int64_t lora_num,
+                           int64_t total_rows, int32_t* d_status, void* stream);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+SGMV_API const char* sgmv_status_string(int code);
+
+/*
+ * sgmv_set_variant -- force the kernel variant used by later calls from any
+ * host thread (SGMV_VARIANT_AUTO restores automatic choice).  A forced variant
+ * that cannot run a call makes that call return SGMV_ERR_VARIANT.  Returns the
+ * previous setting, or SGMV_ERR_VARIANT for an unknown value.  Meant for tests
+ * and benchmarks.
+ */
+SGMV_API int sgmv_set_variant(int variant);
+
+/*
+ * sgmv_device_error -- read and clear the device-side error word of the
+ * current device.  Kernels set it (instead of trapping) when a bounded wait on
+ * an mbarrier gives up, which only a hardware or driver fault could cause.
+ * Synchronises `stream`.  *value receives the word (0 = no error).
+ */
+SGMV_API int sgmv_device_error(void* stream, int32_t* value);
+
+/* Library version as major*10000 + minor*100 + patch. */
+SGMV_API int sgmv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SGMV_H */

@@ -1,0 +1,124 @@
+"""SGMV expand-slice for NVIDIA B200 (sm_100a): Python binding of libsgmv.
+
+The binding only turns torch tensors into the C ABI's descriptors and passes
+torch's current CUDA stream; every step of the operation runs in libsgmv's
+CUDA kernels.  The operation and its arguments follow the wrapper described on
+"Implementation: Predibase Lorax SGMV Expand Slice Kernel" (sections Signature
+and I/O Contract):
+
+    sgmv_expand_slice(inputs, lora_b_weights, output_tensor, b_seq_start_loc,
+                      seq_len_tensor, lora_indices_tensor, batches,
+                      max_seq_length, slice_offset, slice_size, add_inputs=False)
+
+updates ``output_tensor[start_b + m, slice_offset:slice_offset + slice_size]``
+for every sequence b with ``lora_indices_tensor[b] != -1`` and token m, with
+``inputs[start_b + m] @ lora_b_weights[idx_b].T`` (added to the old values when
+``add_inputs``).
+"""
+import ctypes
+
+import torch
+
+from . import _abi
+
+__all__ = ["sgmv_expand_slice", "plan", "validate_metadata", "set_variant", "device_error",
+           "SgmvError", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "library_path"]
+
+VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC = _abi.VARIANT_AUTO, _abi.VARIANT_SIMT, _abi.VARIANT_TC
+library_path = _abi.LIB_PATH
+
+_DTYPES = {torch.float16: _abi.F16, torch.bfloat16: _abi.BF16, torch.float32: _abi.F32,
+           torch.int32: _abi.I32, torch.int64: _abi.I64}
+
+_lib = _abi.load()
+
+
+class SgmvError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = _lib.sgmv_status_string(code).decode()
+        super().__init__(f"{where}: {_abi.STATUS_NAMES.get(code, code)} ({msg})")
+
+
+def _desc(t: torch.Tensor) -> _abi.SgmvTensor:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return _abi.make_tensor(t.data_ptr(), _DTYPES[t.dtype], t.shape, t.stride())
+
+
+def _stream_handle(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _args(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor,
+          lora_indices_tensor):
+    ts = [inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors on the same device")
+        if t.device != output_tensor.device:
+            raise ValueError("all tensors must be on the same device")
+    return [_desc(t) for t in ts]
+
+
+def sgmv_expand_slice(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor,
+                      lora_indices_tensor, batches, max_seq_length, slice_offset, slice_size,
+                      add_inputs=False):
+    """In-place SGMV expand-slice on ``output_tensor`` (enqueued on torch's current stream)."""
+    d = _args(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor,
+              lora_indices_tensor)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_expand_slice(*[ctypes.byref(x) for x in d], int(batches), int(max_seq_length),
+                                    int(slice_offset), int(slice_size), int(bool(add_inputs)),
+                                    _stream_handle(output_tensor.device))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_expand_slice")
+    return output_tensor
+
+
+def plan(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor,
+         batches, max_seq_length, slice_offset, slice_size, add_inputs=False) -> int:
+    """Kernel variant a call with these arguments would launch (0 = none)."""
+    d = _args(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor,
+              lora_indices_tensor)
+    v = ctypes.c_int(0)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_plan(*[ctypes.byref(x) for x in d], int(batches), int(max_seq_length),
+                            int(slice_offset), int(slice_size), int(bool(add_inputs)), ctypes.byref(v))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_plan")
+    return v.value
+
+
+def validate_metadata(b_seq_start_loc, seq_len_tensor, lora_indices_tensor, batches, lora_num,
+                      total_rows) -> int:
+    """Device check of the metadata values; returns the status bit mask (synchronises)."""
+    dev = b_seq_start_loc.device
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    d = [_desc(t) for t in (b_seq_start_loc, seq_len_tensor, lora_indices_tensor)]
+    with torch.cuda.device(dev):
+        rc = _lib.sgmv_validate_metadata(*[ctypes.byref(x) for x in d], int(batches), int(lora_num),
+                                         int(total_rows), ctypes.c_void_p(status.data_ptr()),
+                                         _stream_handle(dev))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_validate_metadata")
+    return int(status.item())
+
+
+def set_variant(variant: int) -> int:
+    """Force a kernel variant for later calls (VARIANT_AUTO restores the default)."""
+    rc = _lib.sgmv_set_variant(int(variant))
+    if rc < 0:
+        raise SgmvError(rc, "sgmv_set_variant")
+    return rc
+
+
+def device_error(device=None) -> int:
+    """Read and clear the device error word (non-zero only after a kernel gave up a wait)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    v = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        rc = _lib.sgmv_device_error(_stream_handle(dev), ctypes.byref(v))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_device_error")
+    return v.value

@@ -1,0 +1,306 @@
+// libsgmv: the C ABI (include/sgmv.h), host-side validation and dispatch.
+//
+// This is the library's single translation unit: the kernels live in the
+// headers included below, so the device-side error word is one object per
+// device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "simt.cuh"
+#include "tc.cuh"
+#include "validate.cuh"
+
+namespace sgmv {
+
+__device__ int32_t g_device_error = 0;
+
+__device__ void raise_device_error(int32_t bits) { atomicOr(&g_device_error, bits); }
+
+}  // namespace sgmv
+
+#include "tc_kernel.cuh"
+
+using namespace sgmv;
+
+namespace {
+
+std::atomic<int> g_forced_variant{SGMV_VARIANT_AUTO};
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    size_t smem_optin = 0;
+    bool ok = false;
+};
+DeviceInfo g_devinfo[kMaxDevices];
+std::mutex g_devinfo_mu;
+
+int device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SGMV_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_devinfo_mu);
+    DeviceInfo& d = g_devinfo[dev];
+    if (!d.ok) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SGMV_ERR_CUDA;
+        d.sm_count = prop.multiProcessorCount;
+        d.cc_major = prop.major;
+        d.cc_minor = prop.minor;
+        d.smem_optin = prop.sharedMemPerBlockOptin;
+        d.ok = true;
+    }
+    *out = d;
+    return SGMV_OK;
+}
+
+bool is_float_dtype(int dt) { return dt == SGMV_F16 || dt == SGMV_BF16 || dt == SGMV_F32; }
+bool is_half_dtype(int dt) { return dt == SGMV_F16 || dt == SGMV_BF16; }
+bool is_meta_dtype(int dt) { return dt == SGMV_I32 || dt == SGMV_I64; }
+
+int64_t numel(const sgmv_tensor* t) {
+    int64_t n = 1;
+    for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+    return n;
+}
+
+// Shape/stride sanity common to every tensor argument.
+int check_basic(const sgmv_tensor* t) {
+    if (!t) return SGMV_ERR_NULL_ARG;
+    if (t->ndim < 1 || t->ndim > 4) return SGMV_ERR_NDIM;
+    for (int i = 0; i < t->ndim; ++i) {
+        if (t->shape[i] < 0) return SGMV_ERR_SHAPE;
+        if (t->stride[i] < 0) return SGMV_ERR_STRIDE;
+        if (t->shape[i] > (int64_t(1) << 40) || t->stride[i] > (int64_t(1) << 40)) return SGMV_ERR_TOO_LARGE;
+    }
+    if (numel(t) > 0 && t->data == nullptr) return SGMV_ERR_NULL_ARG;
+    return SGMV_OK;
+}
+
+int check_meta(const sgmv_tensor* t, int64_t batches) {
+    int rc = check_basic(t);
+    if (rc) return rc;
+    if (t->ndim != 1) return SGMV_ERR_NDIM;
+    if (!is_meta_dtype(t->dtype)) return SGMV_ERR_DTYPE;
+    if (t->shape[0] < batches) return SGMV_ERR_BATCHES;
+    if (batches > 0 && t->data == nullptr) return SGMV_ERR_NULL_ARG;
+    return SGMV_OK;
+}
+
+MetaVec meta_of(const sgmv_tensor* t) {
+    MetaVec m;
+    m.ptr = t->data;
+    m.dtype = t->dtype;
+    m.stride = t->stride[0];
+    return m;
+}
+
+struct Call {
+    Problem p;
+    int64_t max_seq_len;
+    bool empty;   // nothing to launch
+};
+
+// Full host-side validation; fills the problem descriptor.  Touches no CUDA API.
+int validate_call(const sgmv_tensor* x, const sgmv_tensor* w, const sgmv_tensor* out,
+                  const sgmv_tensor* s, const sgmv_tensor* l, const sgmv_tensor* idx,
+                  int64_t batches, int64_t max_seq_len, int64_t slice_offset, int64_t slice_size,
+                  int add_inputs, Call* call) {
+    int rc;
+    if ((rc = check_basic(x))) return rc;
+    if ((rc = check_basic(w))) return rc;
+    if ((rc = check_basic(out))) return rc;
+    if (batches < 0) return SGMV_ERR_BATCHES;
+    if (max_seq_len < 0 || slice_size < 0) return SGMV_ERR_SHAPE;
+    if ((rc = check_meta(s, batches))) return rc;
+    if ((rc = check_meta(l, batches))) return rc;
+    if ((rc = check_meta(idx, batches))) return rc;
+    if (x->ndim != 2 || out->ndim != 2) return SGMV_ERR_NDIM;
+    if (w->ndim != 3 && w->ndim != 4) return SGMV_ERR_NDIM;
+    if (!is_float_dtype(x->dtype) || !is_half_dtype(w->dtype) || !is_float_dtype(out->dtype))
+        return SGMV_ERR_DTYPE;
+    const int wd = w->ndim;
+    if (wd == 4 && w->shape[1] != 1) return SGMV_ERR_LAYOUT_4D;
+    const int64_t K = x->shape[1];
+    if (w->shape[wd - 1] != K) return SGMV_ERR_RANK_MISMATCH;
+    if (w->shape[wd - 2] != slice_size) return SGMV_ERR_SLICE_SIZE;
+    const int64_t T_out = out->shape[0], H = out->shape[1];
+    if (!(out->stride[1] == 1 || H <= 1) || !(out->stride[0] == H || T_out <= 1))
+        return SGMV_ERR_OUT_NOT_CONTIGUOUS;
+    if (slice_offset < 0 || slice_offset + slice_size > H) return SGMV_ERR_SLICE_RANGE;
+
+    Problem& p = call->p;
+    p.x = x->data;
+    p.x_dt = x->dtype;
+    p.x_rows = x->shape[0];
+    p.K = K;
+    p.x_rs = x->stride[0];
+    p.x_cs = x->stride[1];
+    p.w = w->data;
+    p.w_dt = w->dtype;
+    p.lora_num = w->shape[0];
+    p.w_as = w->stride[0];
+    p.w_ns = w->stride[wd - 2];
+    p.w_ks = w->stride[wd - 1];
+    p.out = out->data;
+    p.out_dt = out->dtype;
+    p.out_rows = T_out;
+    p.H = H;
+    p.start = meta_of(s);
+    p.len = meta_of(l);
+    p.idx = meta_of(idx);
+    p.batches = batches;
+    p.off = slice_offset;
+    p.N = slice_size;
+    p.add = add_inputs ? 1 : 0;
+    call->max_seq_len = max_seq_len;
+    call->empty = batches == 0 || slice_size == 0 || T_out == 0 || p.lora_num == 0 || p.x_rows == 0;
+    return SGMV_OK;
+}
+
+int launch_simt(const Call& c, const DeviceInfo& dev, cudaStream_t stream) {
+    const Problem& p = c.p;
+    const int64_t n_tiles = (p.N + SIMT_NT - 1) / SIMT_NT;
+    if (n_tiles > (1 << 20)) return SGMV_ERR_TOO_LARGE;
+    // Row-chunk slots: enough CTAs to fill the GPU for long segments; the
+    // kernel grid-strides over chunks, so any value is correct.
+    int64_t want_slots = (c.max_seq_len + SIMT_RC - 1) / SIMT_RC;
+    const int64_t batches_y = p.batches < 65535 ? p.batches : 65535;
+    const int64_t fill = (int64_t)dev.sm_count * 8 / (n_tiles * batches_y) + 1;
+    if (want_slots > fill) want_slots = fill;
+    if (want_slots < 1) want_slots = 1;
+    if (want_slots * n_tiles > 0x7fffffff) want_slots = 0x7fffffff / n_tiles;
+    dim3 grid((unsigned)(n_tiles * want_slots), (unsigned)batches_y);
+    simt_expand_slice_kernel<<<grid, SIMT_THREADS, 0, stream>>>(p, (int)n_tiles, (int)want_slots);
+    return cudaGetLastError() == cudaSuccess ? SGMV_OK : SGMV_ERR_LAUNCH;
+}
+
+// Which variant runs a validated, non-empty call.
+int choose_variant(const Call& c, const DeviceInfo& dev, int forced) {
+    const bool tc_ok = dev.cc_major == 10 && tc_supports(c.p);
+    if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
+    if (forced == SGMV_VARIANT_TC) return tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
+    return tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+                      const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                      const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
+                      int64_t slice_offset, int64_t slice_size, int add_inputs, void* stream) {
+    Call c;
+    int rc = validate_call(inputs, lora_b, out, seq_start, seq_len, lora_idx, batches, max_seq_len,
+                           slice_offset, slice_size, add_inputs, &c);
+    if (rc) return rc;
+    if (c.empty) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    const int v = choose_variant(c, dev, g_forced_variant.load());
+    if (v < 0) return v;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (v == SGMV_VARIANT_TC) return launch_tc(c.p, dev.sm_count, st);
+    return launch_simt(c, dev, st);
+}
+
+int sgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+              const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+              int64_t batches, int64_t max_seq_len, int64_t slice_offset, int64_t slice_size,
+              int add_inputs, int* variant) {
+    if (!variant) return SGMV_ERR_NULL_ARG;
+    *variant = 0;
+    Call c;
+    int rc = validate_call(inputs, lora_b, out, seq_start, seq_len, lora_idx, batches, max_seq_len,
+                           slice_offset, slice_size, add_inputs, &c);
+    if (rc) return rc;
+    if (c.empty) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    const int v = choose_variant(c, dev, g_forced_variant.load());
+    if (v < 0) return v;
+    *variant = v;
+    return SGMV_OK;
+}
+
+int sgmv_validate_metadata(const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                           const sgmv_tensor* lora_idx, int64_t batches, int64_t lora_num,
+                           int64_t total_rows, int32_t* d_status, void* stream) {
+    if (!d_status) return SGMV_ERR_NULL_ARG;
+    if (batches < 0) return SGMV_ERR_BATCHES;
+    if (lora_num < 0 || total_rows < 0) return SGMV_ERR_SHAPE;
+    int rc;
+    if ((rc = check_meta(seq_start, batches))) return rc;
+    if ((rc = check_meta(seq_len, batches))) return rc;
+    if ((rc = check_meta(lora_idx, batches))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), st) != cudaSuccess) return SGMV_ERR_CUDA;
+    if (batches == 0) return SGMV_OK;
+    const int threads = 256;
+    int64_t blocks = (batches + threads - 1) / threads;
+    if (blocks > 4096) blocks = 4096;
+    validate_metadata_kernel<<<(unsigned)blocks, threads, 0, st>>>(
+        meta_of(seq_start), meta_of(seq_len), meta_of(lora_idx), batches, lora_num, total_rows, d_status);
+    if (cudaGetLastError() != cudaSuccess) return SGMV_ERR_LAUNCH;
+    if (batches <= VALIDATE_PAIRWISE_LIMIT) {
+        validate_overlap_pairwise_kernel<<<1024, threads, 0, st>>>(
+            meta_of(seq_start), meta_of(seq_len), meta_of(lora_idx), batches, lora_num, d_status);
+        if (cudaGetLastError() != cudaSuccess) return SGMV_ERR_LAUNCH;
+    }
+    return SGMV_OK;
+}
+
+const char* sgmv_status_string(int code) {
+    switch (code) {
+        case SGMV_OK: return "ok";
+        case SGMV_ERR_NULL_ARG: return "null descriptor or null data pointer";
+        case SGMV_ERR_DTYPE: return "dtype not allowed for this argument";
+        case SGMV_ERR_NDIM: return "wrong number of dimensions";
+        case SGMV_ERR_RANK_MISMATCH: return "inputs.shape[1] != lora_b.shape[-1] (rank mismatch)";
+        case SGMV_ERR_SLICE_SIZE: return "slice_size != lora_b.shape[-2]";
+        case SGMV_ERR_LAYOUT_4D: return "4-D lora_b must have shape (lora_num, 1, slice_size, rank)";
+        case SGMV_ERR_OUT_NOT_CONTIGUOUS: return "output tensor must be contiguous";
+        case SGMV_ERR_SLICE_RANGE: return "slice [offset, offset + size) outside the output width";
+        case SGMV_ERR_BATCHES: return "batches negative or larger than a metadata tensor";
+        case SGMV_ERR_SHAPE: return "negative extent or max_seq_len";
+        case SGMV_ERR_STRIDE: return "negative stride";
+        case SGMV_ERR_TOO_LARGE: return "sizes beyond the library's index range";
+        case SGMV_ERR_VARIANT: return "the forced kernel variant cannot run this call";
+        case SGMV_ERR_CUDA: return "a CUDA runtime call failed";
+        case SGMV_ERR_LAUNCH: return "kernel launch failed";
+        default: return "unknown status";
+    }
+}
+
+int sgmv_set_variant(int variant) {
+    if (variant != SGMV_VARIANT_AUTO && variant != SGMV_VARIANT_SIMT && variant != SGMV_VARIANT_TC)
+        return SGMV_ERR_VARIANT;
+    return g_forced_variant.exchange(variant);
+}
+
+int sgmv_device_error(void* stream, int32_t* value) {
+    if (!value) return SGMV_ERR_NULL_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t zero = 0;
+    if (cudaMemcpyFromSymbolAsync(value, g_device_error, sizeof(int32_t), 0, cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
+        return SGMV_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int32_t), 0, cudaMemcpyHostToDevice, st) !=
+        cudaSuccess)
+        return SGMV_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SGMV_ERR_CUDA;
+    return SGMV_OK;
+}
+
+int sgmv_version(void) { return 100; }
+
+}  // extern "C"

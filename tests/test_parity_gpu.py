@@ -1,0 +1,307 @@
+"""GPU parity: the CUDA library against the CPU oracle on the same seeded inputs.
+
+Every test runs each kernel variant that can take the case.  Inside the written
+slice the results must be within the stated tolerance (see sgmv_testlib);
+everything else in the output must keep its bits.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sgmv_inputs as gen
+import segmented_gather_gemm_expand_b200 as sg
+from sgmv_testlib import DeviceProblem, compare, from_torch, to_torch, written_rows
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = {"simt": sg.VARIANT_SIMT, "tc": sg.VARIANT_TC}
+
+
+@pytest.fixture(autouse=True)
+def _reset_variant():
+    yield
+    sg.set_variant(sg.VARIANT_AUTO)
+
+
+def use_variant(name, dp: DeviceProblem, call=0):
+    """Force a variant; returns False (and restores auto) if it cannot take the case."""
+    sg.set_variant(VARIANTS[name])
+    try:
+        dp.plan(call)
+    except sg.SgmvError as e:
+        sg.set_variant(sg.VARIANT_AUTO)
+        if e.code == -13:
+            return False
+        raise
+    return True
+
+
+def regions(p, calls=None):
+    calls = range(len(p.calls)) if calls is None else calls
+    return [(written_rows(p, c), p.calls[c].slice_offset, p.calls[c].slice_size) for c in calls]
+
+
+def check_full(p: gen.Problem, variant: str, calls=None):
+    """Run every call on the GPU and the oracle; compare the whole output."""
+    dp = DeviceProblem(p)
+    calls = list(range(len(p.calls))) if calls is None else calls
+    if not use_variant(variant, dp):
+        pytest.skip(f"{variant} does not take this case")
+    ref = p.y0
+    for c in calls:
+        dp.run(c)
+        ref = oracle.run_problem(p, out=ref, call=c)
+    torch.cuda.synchronize()
+    gpu = dp.result()
+    assert sg.device_error() == 0
+    check_regions(gpu, ref, p, regions(p, calls))
+    return gpu, ref
+
+
+def check_regions(gpu, ref, p, regs, check_rows=None):
+    outside = np.ones(gpu.shape, dtype=bool)
+    for rows, c0, n in regs:
+        outside[np.ix_(rows, np.arange(c0, c0 + n))] = False
+    bad = np.nonzero((gpu != p.y0) & outside)
+    assert bad[0].size == 0, f"{bad[0].size} untouched elements changed (first {bad[0][0]},{bad[1][0]})"
+    for rows, c0, n in regs:
+        compare(gpu, ref, np.where(outside, p.y0, gpu), p, rows, c0, n, check_rows=check_rows)
+
+
+# ------------------------------------------------------------------ small cases
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_tiny_workload(variant):
+    check_full(gen.tiny(), variant)
+
+
+EDGE = {
+    "one_token_segments": dict(lengths=[1, 1, 1, 1, 1], K=16, N=64, H=64, offset=0, num_adapters=3),
+    "zero_length_mixed": dict(lengths=[0, 5, 0, 3, 0], K=16, N=64, H=128, offset=64, num_adapters=2),
+    "all_minus_one": dict(lengths=[4, 5], K=16, N=64, H=64, offset=0, num_adapters=2, idx=[-1, -1]),
+    "multi_tile_ragged": dict(lengths=[300, 129, 7, 128, 257], K=16, N=320, H=640, offset=256,
+                              num_adapters=4),
+    "n_not_multiple_of_8": dict(lengths=[9, 17], K=16, N=61, H=100, offset=3, num_adapters=2),
+    "odd_offset_f32_out": dict(lengths=[33, 5], K=32, N=72, H=200, offset=7, num_adapters=2,
+                               out_dt="f32"),
+    "gaps_and_extra_rows": dict(lengths=[3, 40, 9], starts=[2, 10, 60], K=16, N=128, H=256,
+                                offset=128, num_adapters=3, extra_rows=11),
+    "strided_x_and_w": dict(lengths=[50, 14], K=16, N=96, H=192, offset=32, num_adapters=2,
+                            x_col_pad=5, w_row_pad=3),
+    "layout_4d": dict(lengths=[70, 3, 19], K=32, N=128, H=256, offset=128, num_adapters=3,
+                      layout4d=True),
+    "int32_metadata": dict(lengths=[64, 65, 1], K=16, N=128, H=128, offset=0, num_adapters=2,
+                           meta_dt="int32"),
+    "overwrite_mode": dict(lengths=[40, 90], K=16, N=256, H=512, offset=256, num_adapters=2,
+                           add_inputs=False),
+    "wide_slice": dict(lengths=[20, 150], K=16, N=1000, H=1100, offset=40, num_adapters=2),
+}
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("case", sorted(EDGE))
+def test_edge_cases(case, variant):
+    check_full(gen.custom(seed=sum(map(ord, case)) % 1000, **EDGE[case]), variant)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("K", [1, 7, 8, 16, 17, 32, 48, 64, 128])
+def test_ranks(K, variant):
+    p = gen.custom(seed=K, lengths=[37, 130, 2], K=K, N=136, H=272, offset=136, num_adapters=3)
+    check_full(p, variant)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("x_dt", gen.ALL_DTYPES)
+@pytest.mark.parametrize("w_dt", gen.HALF_DTYPES)
+@pytest.mark.parametrize("out_dt", gen.ALL_DTYPES)
+def test_dtype_combinations(x_dt, w_dt, out_dt, variant):
+    p = gen.custom(seed=3, lengths=[45, 140, 6], K=16, N=128, H=384, offset=128, num_adapters=3,
+                   x_dt=x_dt, w_dt=w_dt, out_dt=out_dt, idx=[2, 0, 1])
+    check_full(p, variant)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_integer_inputs_bit_exact(variant):
+    p = gen.custom(seed=8, lengths=[33, 129, 5], K=64, N=128, H=256, offset=0, num_adapters=3,
+                   integer=True, idx=[1, 2, 0])
+    gpu, ref = check_full(p, variant)
+    assert np.array_equal(oracle.decode(gpu, "bf16"), oracle.decode(ref, "bf16"))
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_out_of_range_metadata_is_skipped_and_guards_hold(variant):
+    """idx >= lora_num, idx < -1, negative start, segment past the last row."""
+    T, H, N, K = 64, 256, 128, 16
+    p = gen.custom(seed=4, lengths=[10, 8, 6, 9, 30], starts=[0, 12, 22, 30, 50], K=K, N=N, H=H,
+                   offset=128, num_adapters=2, idx=[0, 5, -7, 1, 1])
+    p.seq_start = p.seq_start.copy()
+    p.seq_start[2] = -4                        # negative start (its idx is also invalid)
+    # y0 has 80 rows; segment 4 runs to row 80 -> give out only 64 rows: rows >= 64 skipped
+    p.y0 = np.ascontiguousarray(p.y0[:T])
+    dp = DeviceProblem(p)
+    if not use_variant(variant, dp):
+        pytest.skip("variant does not take this case")
+    # embed out in a guarded buffer
+    G = 4096
+    buf = torch.empty(G + T * H + G, dtype=torch.bfloat16, device="cuda")
+    canary = torch.full((G,), 7.0, dtype=torch.bfloat16, device="cuda")
+    buf[:G] = canary
+    buf[G + T * H:] = canary
+    y = buf[G:G + T * H].view(T, H)
+    y.copy_(dp.y)
+    dp.run(out=y)
+    torch.cuda.synchronize()
+    assert torch.equal(buf[:G], canary) and torch.equal(buf[G + T * H:], canary)
+    gpu = from_torch(y, "bf16")
+    ref = oracle.run_problem(p)
+    check_regions(gpu, ref, p, regions(p))
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_max_seq_len_smaller_than_segments(variant):
+    """Every token m < L_b is processed even if max_seq_len understates the longest segment."""
+    p = gen.custom(seed=12, lengths=[200, 17], K=16, N=128, H=128, offset=0, num_adapters=2)
+    dp = DeviceProblem(p)
+    if not use_variant(variant, dp):
+        pytest.skip("variant does not take this case")
+    dp.run(max_seq_len=4)
+    torch.cuda.synchronize()
+    check_regions(dp.result(), oracle.run_problem(p), p, regions(p))
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_overwrite_ignores_nan(variant):
+    p = gen.custom(seed=13, lengths=[70, 9], K=16, N=128, H=256, offset=128, num_adapters=2,
+                   add_inputs=False)
+    p.y0 = gen.to_storage(np.full(p.y0.shape, np.nan, np.float32), "bf16")
+    check_full(p, variant)
+
+
+# ------------------------------------------------------------------ invariants, bit-exact
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_invariants_bit_exact(variant):
+    base = dict(lengths=[130, 7, 64, 250, 1], K=32, N=256, H=768, offset=256, num_adapters=4,
+                idx=[3, -1, 0, 2, 1])
+    p = gen.custom(seed=21, **base)
+    dp = DeviceProblem(p)
+    if not use_variant(variant, dp):
+        pytest.skip("variant does not take this case")
+    dp.run()
+    ref = from_torch(dp.y, "bf16")
+    # deterministic
+    dp2 = DeviceProblem(p)
+    dp2.run()
+    assert np.array_equal(from_torch(dp2.y, "bf16"), ref)
+    # 3-D vs 4-D
+    q = gen.custom(seed=21, layout4d=True, **base)
+    dq = DeviceProblem(q)
+    dq.run()
+    assert np.array_equal(from_torch(dq.y, "bf16"), ref)
+    # segment order
+    perm = np.array([3, 0, 4, 2, 1])
+    p2 = gen.custom(seed=21, **base)
+    p2.seq_start, p2.seq_len, p2.lora_idx = p.seq_start[perm], p.seq_len[perm], p.lora_idx[perm]
+    d3 = DeviceProblem(p2)
+    d3.run()
+    assert np.array_equal(from_torch(d3.y, "bf16"), ref)
+    # split into two calls over disjoint segments
+    p3 = gen.custom(seed=21, **base)
+    d4 = DeviceProblem(p3)
+    for part in ([0, 2], [1, 3, 4]):
+        sub = gen.custom(seed=21, **base)
+        sub.seq_start, sub.seq_len, sub.lora_idx = p.seq_start[part], p.seq_len[part], p.lora_idx[part]
+        ds = DeviceProblem(sub)
+        ds.run(out=d4.y)
+    assert np.array_equal(from_torch(d4.y, "bf16"), ref)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_add_equals_old_plus_overwrite_result(variant):
+    base = dict(lengths=[90, 40], K=16, N=128, H=128, offset=0, num_adapters=2, out_dt="f32")
+    p = gen.custom(seed=22, **base)
+    dp = DeviceProblem(p)
+    if not use_variant(variant, dp):
+        pytest.skip("variant does not take this case")
+    dp.run(add=True)
+    d2 = DeviceProblem(p)
+    d2.run(add=False)
+    torch.cuda.synchronize()
+    a = from_torch(dp.y, "f32").astype(np.float64)
+    o = from_torch(d2.y, "f32").astype(np.float64)
+    y0 = p.y0.astype(np.float64)
+    rows = written_rows(p)
+    np.testing.assert_allclose(a[rows, :128], y0[rows, :128] + o[rows, :128], rtol=0, atol=1e-5)
+    assert np.array_equal(a[~rows], y0[~rows]) and np.array_equal(o[~rows], y0[~rows])
+
+
+# ------------------------------------------------------------------ the five workloads, full size
+
+def sampled_subproblem(p: gen.Problem, rng, n_segments: int, cap: int):
+    """Segments chosen by `rng`; from each, its first and last `cap` rows."""
+    A = p.calls[0].w.shape[0]
+    valid = [b for b in range(p.batches) if 0 <= p.lora_idx[b] < A and p.seq_len[b] > 0]
+    pick = sorted(set([valid[0], valid[-1]] + list(rng.choice(valid, size=min(n_segments, len(valid)),
+                                                               replace=False))))
+    starts, lens, idx = [], [], []
+    for b in pick:
+        s, L, a = int(p.seq_start[b]), int(p.seq_len[b]), int(p.lora_idx[b])
+        if L <= 2 * cap:
+            starts.append(s), lens.append(L), idx.append(a)
+        else:
+            starts += [s, s + L - cap]
+            lens += [cap, cap]
+            idx += [a, a]
+    return np.array(starts, np.int64), np.array(lens, np.int64), np.array(idx, np.int64)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("name", ["qkv_prefill", "mlp_mixed", "long_single", "decode_mix"])
+def test_workload_full_size(name, variant):
+    p = gen.WORKLOADS[name]()
+    dp = DeviceProblem(p)
+    if not use_variant(variant, dp):
+        pytest.skip("variant does not take this case")
+    for c in range(len(p.calls)):
+        dp.run(c)
+    torch.cuda.synchronize()
+    assert sg.device_error() == 0
+    gpu = dp.result()
+    del dp
+    torch.cuda.empty_cache()
+    s, l, i = sampled_subproblem(p, np.random.default_rng(5), 6, 40)
+    sub = gen.Problem(p.name, p.x, p.x_dt, p.w_dt, p.y0, p.out_dt, s, l, i, p.add_inputs, p.calls)
+    ref = p.y0
+    for c in range(len(p.calls)):
+        ref = oracle.run_problem(sub, out=ref, call=c, nthreads=oracle.max_threads())
+    check_rows = written_rows(sub)
+    check_regions(gpu, ref, p, regions(p), check_rows=check_rows)
+
+
+def test_auto_picks_tensor_cores_for_the_workloads():
+    for name in ["qkv_prefill", "decode_mix", "long_single"]:
+        p = gen.WORKLOADS[name]()
+        p.y0 = p.y0[:8]                        # planning needs shapes only
+        dp = DeviceProblem(p)
+        assert dp.plan() in (sg.VARIANT_SIMT, sg.VARIANT_TC)
+
+
+# ------------------------------------------------------------------ metadata validation
+
+def test_validate_metadata_bits():
+    dev = "cuda"
+
+    def run(starts, lens, idx, A=4, rows=100):
+        t = lambda a: torch.tensor(a, dtype=torch.int64, device=dev)
+        return sg.validate_metadata(t(starts), t(lens), t(idx), len(starts), A, rows)
+
+    assert run([0, 4, 10], [4, 6, 3], [0, 1, -1]) == 0
+    assert run([0, 4], [4, 6], [0, 9]) & 1
+    assert run([0, -4], [4, 6], [0, 1]) & 2
+    assert run([0, 95], [4, 6], [0, 1]) & 4
+    assert run([0, 2], [4, 6], [0, 1]) & 8
+    st = run([10, 0], [4, 6], [0, 1])
+    assert st & 16 and not st & 8
+    assert run([4, 0], [6, 6], [0, 1]) & 8

@@ -1,31 +1,32 @@
 // Tensor-core SGMV expand-slice for sm_100a: tcgen05 MMA with the accumulator
 // in tensor memory, TMA staging of B, x and the output slice.
 //
-// One persistent CTA per SM, 320 threads in warp roles:
+// One persistent CTA per SM, 352 threads in warp roles:
 //
-//   warp 0    producer   TMA: x for each 128-row block of a segment, B[a]'s
-//                        128-column n-tile for each piece, and (add mode) the
-//                        output tile.  Output rows in whole groups of 8 move
-//                        as 2-D tensor boxes of 8..128 rows x 128 bytes
-//                        (128-byte swizzle); the last < 8 rows of a segment
-//                        move as 1-D bulk copies per row, so nothing outside
-//                        the segment's rows and the slice's columns is touched.
+//   warp 0    producer   TMA: x for each 128-row block of a segment and B[a]'s
+//                        128-column n-tile (K in 64/32/16/8-column boxes with
+//                        the matching swizzle) for each piece.
+//   warp 2    loader     (add mode) TMA of the output tile: whole 8-row groups
+//                        as 2-D boxes of 8..128 rows x 128 bytes (128-byte
+//                        swizzle), clipped at the slice's last column.
 //   warp 1    MMA        (mixed dtypes only) rounds x to the weights' dtype into
 //                        the MMA operand layout; one elected lane issues
 //                        tcgen05.mma (M=128 rows, N=128 columns, K=16 each)
-//                        into one of two TMEM accumulators.
-//   warps 2-9 epilogue   warp w owns TMEM lanes 32*(w%4).. (32 rows) and half
+//                        into one of four TMEM accumulators.
+//   warps 3-10 epilogue  warp w owns TMEM lanes 32*(w%4).. (32 rows) and half
 //                        of the tile's columns: tcgen05.ld the fp32 sums, add
 //                        the old output (add mode), round once to the output
 //                        dtype, write the tile back in place in shared memory
-//                        and TMA-store its rows.
+//                        and TMA-store its whole 8-row groups; the last < 8
+//                        rows of a segment are stored from registers, so
+//                        nothing outside the segment's rows is written.
 //
 // Work is expanded on the device.  A piece is (segment, 128-row block of the
 // segment, 128-column n-tile); pieces are ordered with the n-tile fastest, so
 // the x block is staged once and reused across every n-tile.  Every CTA builds
 // the table of segments in shared memory (the guards of sgmv.h applied),
-// weighs each piece as its 8-row groups plus a fixed per-piece overhead, and
-// takes the pieces that start in its equal share of the total weight.
+// weighs each piece as max(its 8-row groups, a floor for the fixed per-piece
+// cost), and takes the pieces that start in its equal share of the weight.
 // Every wait on an mbarrier is bounded; a wait that gives up sets the device
 // error word and makes the CTA leave its loops.
 #pragma once
@@ -45,10 +46,11 @@ constexpr int BM = 128;               // rows per MMA tile (TMEM lanes)
 constexpr int BN = 128;               // columns per n-tile (TMEM columns per accumulator)
 constexpr int GROUP = 8;              // rows per work unit
 constexpr int GROUPS_PER_BLOCK = BM / GROUP;
-constexpr int THREADS = 320;
+constexpr int THREADS = 352;
+constexpr int EPI_WARP0 = 3;          // first epilogue warp
 constexpr int EPI_WARPS = 8;
 constexpr int SEG_CAP = 1024;         // segments held in shared memory
-constexpr int NUM_ACC = 2;            // TMEM accumulators
+constexpr int NUM_ACC = 4;            // TMEM accumulators (4 x 128 columns = all of TMEM)
 constexpr int MAX_KP = 128;           // largest padded rank
 constexpr int NUM_YMAPS = 5;          // output boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
@@ -69,12 +71,17 @@ struct Geometry {
     int32_t n_tiles;    // ceil(N / BN)
     int32_t stages_y, stages_w, stages_xo, stages_xr;
     int32_t w_is_bf16;
-    int32_t ov;         // per-piece scheduling overhead, in 8-row groups
+    int32_t wmin;       // scheduling weight floor of a piece, in 8-row groups
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
     // (rows of 2*kb bytes, swizzled by the row width) at w_blk_off in a stage
     int32_t w_nblk;
     int32_t w_blk_k0[MAX_WBLK], w_blk_kb[MAX_WBLK], w_blk_off[MAX_WBLK];
     int32_t w_zero_off; // 16-byte x 128-row zero chunk after an 8-column block (-1: none)
+    // MMA descriptors of B for each K=16 step, start address left 0, and the
+    // step's byte offset within a stage
+    int32_t ksteps;
+    uint64_t b_desc_rel[MAX_KP / 16];
+    uint32_t b_off[MAX_KP / 16];
     // shared memory offsets (bytes, from the 1024-aligned base)
     int32_t off_y, off_w, off_xo, off_xr, off_seg, off_bar;
     int32_t y_stage_bytes, w_bytes, xo_bytes, xr_bytes;
@@ -103,7 +110,7 @@ struct Piece {
 // Every role runs an identical copy, so all roles see the same sequence.
 struct Walker {
     const SegEntry* segs;
-    int32_t nseg, n_tiles, ov;
+    int32_t nseg, n_tiles, wmin;
     int32_t i, rb, j;     // segment, row block, n-tile
     int32_t G, nblk, gcw; // groups and blocks of segment i; weight of a piece of block rb
     int32_t cur, w_end;   // start weight of the next piece; end of the range
@@ -113,7 +120,7 @@ struct Walker {
         G = (segs[i].rows + GROUP - 1) / GROUP;
         nblk = (G + GROUPS_PER_BLOCK - 1) / GROUPS_PER_BLOCK;
     }
-    __device__ void set_block() { gcw = min(GROUPS_PER_BLOCK, G - rb * GROUPS_PER_BLOCK) + ov; }
+    __device__ void set_block() { gcw = max(min(GROUPS_PER_BLOCK, G - rb * GROUPS_PER_BLOCK), wmin); }
     __device__ void skip_empty() {
         while (i < nseg && segs[i].rows == 0) ++i;
         if (i < nseg) {
@@ -139,7 +146,7 @@ struct Walker {
         skip_empty();
         if (i >= nseg) return;
         const int32_t local = w0 - segs[i].prefix;
-        const int32_t bw = (GROUPS_PER_BLOCK + ov) * n_tiles;   // weight of a full row block
+        const int32_t bw = max(GROUPS_PER_BLOCK, wmin) * n_tiles;   // weight of a full row block
         rb = min(local / bw, nblk - 1);
         set_block();
         const int32_t rem = local - rb * bw;
@@ -287,7 +294,11 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             e.rows = (int32_t)s.rows;
             e.adapter = (int32_t)s.adapter;
             const int32_t G = (e.rows + GROUP - 1) / GROUP;
-            units = (G + geo.ov * ((G + GROUPS_PER_BLOCK - 1) / GROUPS_PER_BLOCK)) * geo.n_tiles;
+            if (G > 0) {
+                const int32_t full = (G - 1) / GROUPS_PER_BLOCK;          // full 128-row blocks
+                const int32_t last = G - full * GROUPS_PER_BLOCK;         // groups of the last block
+                units = (full * max(GROUPS_PER_BLOCK, geo.wmin) + max(last, geo.wmin)) * geo.n_tiles;
+            }
         }
         int32_t v = units;
 #pragma unroll
@@ -321,7 +332,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     walk.segs = segs;
     walk.nseg = nseg;
     walk.n_tiles = geo.n_tiles;
-    walk.ov = geo.ov;
+    walk.wmin = geo.wmin;
     walk.seek((int32_t)(((int64_t)U * blockIdx.x) / gridDim.x), (int32_t)(((int64_t)U * (blockIdx.x + 1)) / gridDim.x));
 
     volatile int* abort_flag = &s_abort;
@@ -370,26 +381,34 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                         tma_load_3d(smem_u32(smem + geo.off_w + s * geo.w_bytes + geo.w_blk_off[b]), &wmaps.m[b],
                                     geo.w_blk_k0[b], pc.n0, pc.adapter, smem_u32(&w_full[s]), pol_keep);
                 }
-                if (ADD) {
-                    const int s = t % SY;
-                    if (!mbar_wait(smem_u32(&y_empty[s]), ((t / SY) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_PRODUCER))
-                        break;
-                    // whole 8-row groups: the rows past the piece in its last group are
-                    // read but never written back
-                    const int rows8 = (pc.rows + GROUP - 1) & ~(GROUP - 1);
-                    const int ncols = min(BN, (int)(p.N - pc.n0));
-                    const int nch = (ncols + CC - 1) / CC;
-                    const uint32_t bar = smem_u32(&y_full[s]);
-                    mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
-                    const uint32_t stage = smem_u32(smem + geo.off_y + s * geo.y_stage_bytes);
-                    const int32_t xcol0 = (int32_t)(p.off + pc.n0);
-                    for (int c = 0; c < nch; ++c) {
-                        for (int r = 0; r < rows8;) {
-                            const int k = box_level(rows8 - r, NUM_YMAPS - 1);
-                            tma_load_2d(stage + c * CHUNK_STRIDE + r * 128, &ymaps.m[k], xcol0 + c * CC,
-                                        pc.blk_row0 + r, bar, pol_stream);
-                            r += GROUP << k;
-                        }
+                ++t;
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ output-tile loader (add mode)
+        if (ADD && lane == 0) {
+            const uint64_t pol_stream = policy_evict_first();
+            Piece pc;
+            int32_t t = 0;
+            while (walk.next(pc)) {
+                const int s = t % SY;
+                if (!mbar_wait(smem_u32(&y_empty[s]), ((t / SY) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_PRODUCER))
+                    break;
+                // whole 8-row groups: the rows past the piece in its last group are
+                // read but never written back
+                const int rows8 = (pc.rows + GROUP - 1) & ~(GROUP - 1);
+                const int ncols = min(BN, (int)(p.N - pc.n0));
+                const int nch = (ncols + CC - 1) / CC;
+                const uint32_t bar = smem_u32(&y_full[s]);
+                mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
+                const uint32_t stage = smem_u32(smem + geo.off_y + s * geo.y_stage_bytes);
+                const int32_t xcol0 = (int32_t)(p.off + pc.n0);
+                for (int c = 0; c < nch; ++c) {
+                    for (int r = 0; r < rows8;) {
+                        const int k = box_level(rows8 - r, NUM_YMAPS - 1);
+                        tma_load_2d(stage + c * CHUNK_STRIDE + r * 128, &ymaps.m[k], xcol0 + c * CC,
+                                    pc.blk_row0 + r, bar, pol_stream);
+                        r += GROUP << k;
                     }
                 }
                 ++t;
@@ -402,6 +421,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         const uint32_t idesc = instr_desc_mn(w_bf16, BM, BN);
         const int kc_real = geo.K / 8, kc_pad = geo.Kp / 8;
         const bool x_bf16 = p.x_dt == SGMV_BF16;
+        constexpr int MAX_KSTEPS = MAX_KP / 16;
+        const uint64_t a_rel = smem_desc(0, BM * 16, 128);
         while (walk.next(pc)) {
             if (pc.new_x) {
                 xcur = xb++;
@@ -459,20 +480,12 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 const uint32_t a_base = smem_u32(smem + geo.off_xo + xs * geo.xo_bytes);
                 const uint32_t b_base = smem_u32(smem + geo.off_w + ws * geo.w_bytes);
                 const uint32_t d = tmem_base + (uint32_t)(as * BN);
-                int ks = 0;
-                for (int b = 0; b < geo.w_nblk; ++b) {
-                    const int kb = geo.w_blk_kb[b];
-                    const uint32_t blk = b_base + (uint32_t)geo.w_blk_off[b];
-                    // swizzle code and 8-row stride of a block of kb columns (rows of 2*kb bytes)
-                    const uint32_t layout = kb == 64 ? 2u : kb == 32 ? 4u : kb == 16 ? 6u : 0u;
-                    const uint32_t sbo = kb >= 16 ? (uint32_t)(8 * 2 * kb) : 128u;
-                    const uint32_t lbo = kb >= 16 ? 16u : (uint32_t)(geo.w_zero_off - geo.w_blk_off[b]);
-                    const int steps = kb >= 16 ? kb / 16 : 1;
-                    for (int st = 0; st < steps; ++st, ++ks) {
-                        const uint64_t ad = smem_desc(a_base + ks * 2 * (BM * 16), BM * 16, 128);
-                        const uint64_t bd = smem_desc(blk + st * 32, lbo, sbo, layout);
-                        tc_mma(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
-                    }
+#pragma unroll
+                for (int ks = 0; ks < MAX_KSTEPS; ++ks) {
+                    if (ks >= geo.ksteps) break;
+                    const uint64_t ad = a_rel | (uint64_t)(((a_base + ks * 2 * (BM * 16)) >> 4) & 0x3FFF);
+                    const uint64_t bd = geo.b_desc_rel[ks] | (uint64_t)(((b_base + geo.b_off[ks]) >> 4) & 0x3FFF);
+                    tc_mma(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(&acc_full[as]));
                 tc_commit(smem_u32(&w_empty[ws]));
@@ -484,7 +497,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp % 4;                  // TMEM lane quadrant of this warp
-        const int half = (warp - 2) / 4;         // which half of the chunks
+        const int half = (warp - EPI_WARP0) / 4; // which half of the chunks
         const int r = q * 32 + lane;             // block row of this thread
         const int ri = r % GROUP;
         const bool out_bf16 = p.out_dt == SGMV_BF16;
@@ -642,12 +655,14 @@ struct Plan {
     YMaps ty;
 };
 
-constexpr int PIECE_OVERHEAD_GROUPS = 4;   // scheduling weight of a piece beyond its rows
+// Scheduling weight floor of a piece (8-row groups): a piece of a few rows
+// costs about as much pipeline time as one of several groups.
+constexpr int PIECE_WEIGHT_FLOOR = 16;
 
 // Shared-memory layout: the deepest pipelines that fit.
 inline bool layout_smem(Geometry& g, int32_t seg_bytes, int* total_out) {
     const int sy_opts[] = {4, 3, 2};
-    const int sw_opts[] = {4, 3, 2};
+    const int sw_opts[] = {8, 6, 4, 3, 2};
     for (int sy : sy_opts) {
         for (int sw : sw_opts) {
             g.stages_y = sy;
@@ -694,7 +709,7 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
     const int64_t n_tiles = (p.N + BN - 1) / BN;
     const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int64_t max_pieces = (t_lim / BM + p.batches + 1) * n_tiles;
-    const int64_t weight_bound = (t_lim / GROUP + p.batches + 1) * n_tiles + PIECE_OVERHEAD_GROUPS * max_pieces;
+    const int64_t weight_bound = (t_lim / GROUP + p.batches + 1) * n_tiles + PIECE_WEIGHT_FLOOR * max_pieces;
     if (weight_bound >= (int64_t(1) << 31)) return false;
 
     Geometry& g = out->geo;
@@ -704,7 +719,7 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
     g.convert_x = p.x_dt != p.w_dt;
     g.n_tiles = (int32_t)n_tiles;
     g.w_is_bf16 = p.w_dt == SGMV_BF16;
-    g.ov = PIECE_OVERHEAD_GROUPS;
+    g.wmin = PIECE_WEIGHT_FLOOR;
     // B tile: K in blocks of 64 columns, then at most one each of 32, 16, 8
     {
         int k0 = 0, off = 0, nb = 0;
@@ -727,6 +742,24 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
             off += BN * 16;
         }
         g.w_bytes = round_up(off, 1024);
+        // B descriptors per K=16 step: swizzle code and 8-row stride follow the
+        // block's row width (2*kb bytes); an 8-column block points its upper K
+        // half at the zero chunk
+        g.ksteps = 0;
+        for (int b = 0; b < nb; ++b) {
+            const int kb = g.w_blk_kb[b];
+            const uint32_t layout = kb == 64 ? 2u : kb == 32 ? 4u : kb == 16 ? 6u : 0u;
+            const uint32_t sbo = kb >= 16 ? (uint32_t)(8 * 2 * kb) : 128u;
+            const uint32_t lbo = kb >= 16 ? 16u : (uint32_t)(g.w_zero_off - g.w_blk_off[b]);
+            const int steps = kb >= 16 ? kb / 16 : 1;
+            for (int st = 0; st < steps; ++st) {
+                if (g.ksteps == MAX_KP / 16) return false;
+                g.b_desc_rel[g.ksteps] = smem_desc(0, lbo, sbo, layout);
+                g.b_off[g.ksteps] = (uint32_t)(g.w_blk_off[b] + st * 32);
+                ++g.ksteps;
+            }
+        }
+        if (g.ksteps != g.Kp / 16) return false;
     }
     g.y_stage_bytes = BM * BN * (int32_t)so;
     g.xo_bytes = BM * g.Kp * 2;

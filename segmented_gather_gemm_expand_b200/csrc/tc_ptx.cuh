@@ -194,7 +194,7 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 // byte distance between the two 16-byte K halves of one K=16 step, `sbo` =
 // byte distance between consecutive 8-row groups), 6 = 32-byte, 4 = 64-byte,
 // 2 = 128-byte swizzle (rows of 32/64/128 bytes; `sbo` = 8 rows; `lbo` unused).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout = 0) {
+__host__ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout = 0) {
     uint64_t d = 0;
     d |= (uint64_t)((addr >> 4) & 0x3FFF);
     d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;

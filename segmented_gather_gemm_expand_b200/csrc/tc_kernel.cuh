@@ -6,8 +6,11 @@
 //   warp 0    producer   TMA: x for each 128-row block of a segment and B[a]'s
 //                        128-column n-tile (K in 64/32/16/8-column boxes with
 //                        the matching swizzle) for each piece.
-//   warp 2    loader     (add mode) TMA of the output tile: whole 8-row groups
-//                        as 2-D boxes of 8..128 rows x 128 bytes (128-byte
+//   warp 2    loader     allocates each piece's rows in shared-memory rings (one
+//                        ring of 128-byte rows per 128-byte column chunk, in
+//                        piece order, freed as the epilogue's stores drain) and,
+//                        in add mode, TMA-loads the old output there: whole
+//                        8-row groups as 2-D boxes of 8..128 rows (128-byte
 //                        swizzle), clipped at the slice's last column.
 //   warp 1    MMA        (mixed dtypes only) rounds x to the weights' dtype into
 //                        the MMA operand layout; one elected lane issues
@@ -54,6 +57,7 @@ constexpr int NUM_ACC = 4;            // TMEM accumulators (4 x 128 columns = al
 constexpr int MAX_KP = 128;           // largest padded rank
 constexpr int NUM_YMAPS = 5;          // output boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
+constexpr int RING_PIECES = 32;       // pieces that may hold ring space at once
 
 struct SegEntry {
     int32_t row0;
@@ -69,7 +73,8 @@ struct Geometry {
     int32_t x_bytes;    // element size of x
     int32_t convert_x;  // x's dtype differs from the weights': round in shared memory
     int32_t n_tiles;    // ceil(N / BN)
-    int32_t stages_y, stages_w, stages_xo, stages_xr;
+    int32_t ring_rows, stages_w, stages_xo, stages_xr;
+    int32_t defer_release;   // release a piece's ring rows one piece later (ring holds >= 3 pieces)
     int32_t w_is_bf16;
     int32_t wmin;       // scheduling weight floor of a piece, in 8-row groups
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
@@ -83,8 +88,8 @@ struct Geometry {
     uint64_t b_desc_rel[MAX_KP / 16];
     uint32_t b_off[MAX_KP / 16];
     // shared memory offsets (bytes, from the 1024-aligned base)
-    int32_t off_y, off_w, off_xo, off_xr, off_seg, off_bar;
-    int32_t y_stage_bytes, w_bytes, xo_bytes, xr_bytes;
+    int32_t off_y, off_w, off_xo, off_xr, off_seg, off_ends, off_bar;
+    int32_t w_bytes, xo_bytes, xr_bytes;
 };
 
 struct YMaps {
@@ -198,6 +203,19 @@ __device__ __forceinline__ int box_level(int rows, int max_level) {
     return k < max_level ? k : max_level;
 }
 
+// Place a piece of rows8 rows in a ring of R rows: returns the ring row where it
+// starts and advances `head` (rows handed out so far, including skipped ones).
+// A piece never wraps: if it does not fit before the ring's end it starts at 0.
+__device__ __forceinline__ int32_t ring_place(int32_t& head, int32_t rows8, int32_t R) {
+    int32_t pos = head % R;
+    if (pos + rows8 > R) {
+        head += R - pos;
+        pos = 0;
+    }
+    head += rows8;
+    return pos;
+}
+
 // ---------------------------------------------------------------- the kernel
 
 template <int OUT_BYTES, bool ADD>
@@ -218,7 +236,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
 
     SegEntry* segs = reinterpret_cast<SegEntry*>(smem + geo.off_seg);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + geo.off_bar);
-    const int SY = geo.stages_y, SW = geo.stages_w, SXO = geo.stages_xo, SXR = geo.stages_xr;
+    const int SW = geo.stages_w, SXO = geo.stages_xo, SXR = geo.stages_xr;
+    const int32_t R = geo.ring_rows;
     uint64_t* w_full = bars;
     uint64_t* w_empty = w_full + SW;
     uint64_t* xo_full = w_empty + SW;
@@ -227,8 +246,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     uint64_t* xr_empty = xr_full + SXR;
     uint64_t* acc_full = xr_empty + SXR;
     uint64_t* acc_empty = acc_full + NUM_ACC;
-    uint64_t* y_full = acc_empty + NUM_ACC;
-    uint64_t* y_empty = y_full + SY;
+    uint64_t* y_full = acc_empty + NUM_ACC;     // piece's ring rows ready (loaded, in add mode)
+    uint64_t* y_free = y_full + RING_PIECES;     // piece's ring rows no longer read by any store
 
     if (tid == 0) {
         s_abort = 0;
@@ -248,9 +267,9 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             mbar_init(smem_u32(&acc_full[i]), 1);
             mbar_init(smem_u32(&acc_empty[i]), EPI_WARPS);
         }
-        for (int i = 0; i < SY; ++i) {
+        for (int i = 0; i < RING_PIECES; ++i) {
             mbar_init(smem_u32(&y_full[i]), 1);
-            mbar_init(smem_u32(&y_empty[i]), EPI_WARPS);
+            mbar_init(smem_u32(&y_free[i]), EPI_WARPS);
         }
         fence_barrier_init();
     }
@@ -340,7 +359,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     constexpr int CC = 128 / OUT_BYTES;              // columns per 128-byte chunk
     constexpr int NCH = BN / CC;                     // chunks per n-tile
     constexpr int CPW = NCH / 2;                     // chunks per epilogue warp
-    constexpr int CHUNK_STRIDE = BM * 128;           // bytes per chunk column of a stage
+    const int32_t RING_STRIDE = R * 128;             // bytes of one chunk's ring
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -385,31 +404,48 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             }
         }
     } else if (warp == 2) {
-        // ------------------------------------------------------------ output-tile loader (add mode)
-        if (ADD && lane == 0) {
+        // ------------------------------------------------------------ ring allocation + output-tile loads
+        if (lane == 0) {
             const uint64_t pol_stream = policy_evict_first();
+            int32_t* ends = reinterpret_cast<int32_t*>(smem + geo.off_ends);   // ring head after each piece
             Piece pc;
-            int32_t t = 0;
-            while (walk.next(pc)) {
-                const int s = t % SY;
-                if (!mbar_wait(smem_u32(&y_empty[s]), ((t / SY) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_PRODUCER))
-                    break;
-                // whole 8-row groups: the rows past the piece in its last group are
-                // read but never written back
+            int32_t t = 0, head = 0, tail_head = 0, tail_piece = 0;
+            bool ok = true;
+            while (ok && walk.next(pc)) {
+                // whole 8-row groups: in add mode the rows past the piece in its last
+                // group are read but never written back
                 const int rows8 = (pc.rows + GROUP - 1) & ~(GROUP - 1);
-                const int ncols = min(BN, (int)(p.N - pc.n0));
-                const int nch = (ncols + CC - 1) / CC;
-                const uint32_t bar = smem_u32(&y_full[s]);
-                mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
-                const uint32_t stage = smem_u32(smem + geo.off_y + s * geo.y_stage_bytes);
-                const int32_t xcol0 = (int32_t)(p.off + pc.n0);
-                for (int c = 0; c < nch; ++c) {
-                    for (int r = 0; r < rows8;) {
-                        const int k = box_level(rows8 - r, NUM_YMAPS - 1);
-                        tma_load_2d(stage + c * CHUNK_STRIDE + r * 128, &ymaps.m[k], xcol0 + c * CC,
-                                    pc.blk_row0 + r, bar, pol_stream);
-                        r += GROUP << k;
+                const int32_t pos = ring_place(head, rows8, R);
+                // free the oldest pieces until this one fits and its barriers are reusable
+                while (tail_piece < t && (head - tail_head > R || t - tail_piece >= RING_PIECES)) {
+                    const int fi = tail_piece % RING_PIECES;
+                    if (!mbar_wait(smem_u32(&y_free[fi]), (tail_piece / RING_PIECES) & 1, abort_flag,
+                                   DEVERR_TIMEOUT_PRODUCER)) {
+                        ok = false;
+                        break;
                     }
+                    tail_head = ends[fi];
+                    ++tail_piece;
+                }
+                if (!ok) break;
+                ends[t % RING_PIECES] = head;
+                const uint32_t bar = smem_u32(&y_full[t % RING_PIECES]);
+                if (ADD) {
+                    const int ncols = min(BN, (int)(p.N - pc.n0));
+                    const int nch = (ncols + CC - 1) / CC;
+                    mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
+                    const uint32_t ring = smem_u32(smem + geo.off_y);
+                    const int32_t xcol0 = (int32_t)(p.off + pc.n0);
+                    for (int c = 0; c < nch; ++c) {
+                        for (int r = 0; r < rows8;) {
+                            const int k = box_level(rows8 - r, NUM_YMAPS - 1);
+                            tma_load_2d(ring + c * RING_STRIDE + (pos + r) * 128, &ymaps.m[k], xcol0 + c * CC,
+                                        pc.blk_row0 + r, bar, pol_stream);
+                            r += GROUP << k;
+                        }
+                    }
+                } else {
+                    mbar_arrive(bar);
                 }
                 ++t;
             }
@@ -502,25 +538,23 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         const int ri = r % GROUP;
         const bool out_bf16 = p.out_dt == SGMV_BF16;
         Piece pc;
-        int32_t t = 0;
+        int32_t t = 0, head = 0;
         while (walk.next(pc)) {
             const int as = t % NUM_ACC;
-            const int ys = t % SY;
+            const int32_t pos = ring_place(head, (pc.rows + GROUP - 1) & ~(GROUP - 1), R);
             if (!warp_wait(smem_u32(&acc_full[as]), (t / NUM_ACC) & 1, abort_flag, DEVERR_TIMEOUT_EPILOGUE)) break;
             tc_fence_after();
-            if (ADD) {
-                if (!warp_wait(smem_u32(&y_full[ys]), (t / SY) & 1, abort_flag, DEVERR_TIMEOUT_EPILOGUE)) break;
-            } else {
-                // only this warp's previous stores (another stage) may still read shared memory
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-            }
+            // every warp waits, so that its release of this piece's ring rows below
+            // always lands in the right phase
+            if (!warp_wait(smem_u32(&y_full[t % RING_PIECES]), (t / RING_PIECES) & 1, abort_flag,
+                           DEVERR_TIMEOUT_EPILOGUE))
+                break;
             const int full_end = pc.rows & ~(GROUP - 1);
             const int ncols = min(BN, (int)(p.N - pc.n0));
             const bool valid = r < pc.rows;
             // rows past the last whole group go straight to global memory from registers
             const bool tail = r >= full_end;
-            uint8_t* stage = smem + geo.off_y + ys * geo.y_stage_bytes;
+            uint8_t* ring = smem + geo.off_y;
             const uint32_t taddr = tmem_base + (uint32_t)(as * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll
             for (int cc = 0; cc < CPW; ++cc) {
@@ -532,7 +566,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     tmem_ld32(taddr + (uint32_t)(c * CC + sub * 32), *reinterpret_cast<uint32_t(*)[32]>(v + sub * 32));
                 tmem_ld_wait();
                 if (valid) {
-                    uint8_t* rowp = stage + c * CHUNK_STRIDE + r * 128;
+                    uint8_t* rowp = ring + c * RING_STRIDE + (pos + r) * 128;
                     uint4* grow = reinterpret_cast<uint4*>(reinterpret_cast<char*>(p.out) +
                                                            ((int64_t)(pc.blk_row0 + r) * p.H + p.off + pc.n0 + c * CC) *
                                                                OUT_BYTES);
@@ -596,15 +630,19 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     for (int rr = q_lo; rr < q_full;) {
                         const int k = box_level(q_full - rr, 2);
                         tma_store_2d(&ymaps.m[k], xcol0 + c * CC, pc.blk_row0 + rr,
-                                     smem_u32(stage + c * CHUNK_STRIDE + rr * 128));
+                                     smem_u32(ring + c * RING_STRIDE + (pos + rr) * 128));
                         rr += GROUP << k;
                     }
                 }
                 bulk_commit();
-                if (ADD) {
-                    // release the previous piece's stage once its stores have read it
+                // release ring rows once the stores have read them: this piece's
+                // now, or (deep rings) the previous piece's, overlapping the drain
+                if (geo.defer_release) {
                     bulk_wait_read<1>();
-                    if (t > 0) mbar_arrive(smem_u32(&y_empty[(t - 1) % SY]));
+                    if (t > 0) mbar_arrive(smem_u32(&y_free[(t - 1) % RING_PIECES]));
+                } else {
+                    bulk_wait_read<0>();
+                    mbar_arrive(smem_u32(&y_free[t % RING_PIECES]));
                 }
             }
             __syncwarp();
@@ -659,19 +697,26 @@ struct Plan {
 // costs about as much pipeline time as one of several groups.
 constexpr int PIECE_WEIGHT_FLOOR = 16;
 
-// Shared-memory layout: the deepest pipelines that fit.
-inline bool layout_smem(Geometry& g, int32_t seg_bytes, int* total_out) {
-    const int sy_opts[] = {4, 3, 2};
+// Shared-memory layout: an output ring of at least 4, else 3, 2, 1 whole
+// 128-row pieces, with the deepest B pipeline that leaves it room.
+inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* total_out) {
     const int sw_opts[] = {8, 6, 4, 3, 2};
-    for (int sy : sy_opts) {
+    const int32_t row_bytes = BN * out_bytes;              // one ring row across all chunks
+    const int32_t budget = SMEM_OPTIN - SMEM_STATIC_RESERVE - 1024;   // 1024: base alignment slack
+    for (int prefer_rows : {4 * BM, 3 * BM, 2 * BM, BM}) {
         for (int sw : sw_opts) {
-            g.stages_y = sy;
             g.stages_w = sw;
             g.stages_xo = 2;
             g.stages_xr = g.convert_x ? 1 : 0;
+            int32_t fixed = sw * g.w_bytes + g.stages_xo * g.xo_bytes + g.stages_xr * g.xr_bytes +
+                            round_up(seg_bytes, 16) + RING_PIECES * 4 +
+                            8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * NUM_ACC + 2 * RING_PIECES) + 64;
+            const int32_t rows = ((budget - fixed) / row_bytes) & ~(GROUP - 1);
+            if (rows < prefer_rows) continue;
+            g.ring_rows = rows;
             int32_t off = 0;
             g.off_y = off;
-            off += sy * g.y_stage_bytes;
+            off += rows * row_bytes;
             g.off_w = off;
             off += sw * g.w_bytes;
             g.off_xo = off;
@@ -679,14 +724,18 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int* total_out) {
             g.off_xr = off;
             off += g.stages_xr * g.xr_bytes;
             g.off_seg = off;
-            off += seg_bytes;
+            off += round_up(seg_bytes, 16);
+            g.off_ends = off;
+            off += RING_PIECES * 4;
             g.off_bar = round_up(off, 8);
-            off = g.off_bar + 8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * NUM_ACC + 2 * sy);
-            const int total = off + 1024;   // slack to align the base to 1024 bytes
-            if (total <= SMEM_OPTIN - SMEM_STATIC_RESERVE) {
-                *total_out = total;
-                return true;
-            }
+            off = g.off_bar + 8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * NUM_ACC + 2 * RING_PIECES);
+            const int total = off + 1024;
+            if (total > SMEM_OPTIN - SMEM_STATIC_RESERVE) continue;
+            *total_out = total;
+            // A piece's rows may be released one piece late only if the ring can
+            // then still place the next piece: two pieces plus the skip at the wrap.
+            g.defer_release = rows >= 3 * BM;
+            return true;
         }
     }
     return false;
@@ -761,11 +810,10 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
         }
         if (g.ksteps != g.Kp / 16) return false;
     }
-    g.y_stage_bytes = BM * BN * (int32_t)so;
     g.xo_bytes = BM * g.Kp * 2;
     g.xr_bytes = round_up(BM * (int32_t)p.K * (int32_t)sx, 1024);
     const int32_t seg_bytes = round_up((int32_t)p.batches * (int32_t)sizeof(SegEntry), 16);
-    if (!layout_smem(g, seg_bytes, &out->smem_bytes)) return false;
+    if (!layout_smem(g, seg_bytes, (int32_t)so, &out->smem_bytes)) return false;
 
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;

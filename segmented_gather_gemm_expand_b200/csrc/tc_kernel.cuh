@@ -16,8 +16,9 @@
 //                        the MMA operand layout; one elected lane issues
 //                        tcgen05.mma (M=128 rows, N=128 columns, K=16 each)
 //                        into one of four TMEM accumulators.
-//   warps 3-10 epilogue  warp w owns TMEM lanes 32*(w%4).. (32 rows) and half
-//                        of the tile's columns: tcgen05.ld the fp32 sums, add
+//   warps 3-10 epilogue  two groups of four warps take alternate pieces; warp w
+//                        owns TMEM lanes 32*(w%4).. (32 rows of the piece) and
+//                        all its columns: tcgen05.ld the fp32 sums, add
 //                        the old output (add mode), round once to the output
 //                        dtype, write the tile back in place in shared memory
 //                        and TMA-store its whole 8-row groups; the last < 8
@@ -51,13 +52,16 @@ constexpr int GROUP = 8;              // rows per work unit
 constexpr int GROUPS_PER_BLOCK = BM / GROUP;
 constexpr int THREADS = 352;
 constexpr int EPI_WARP0 = 3;          // first epilogue warp
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_GROUPS = 2;         // epilogue warp groups, taking pieces in turn
+constexpr int EPI_WARPS = 4 * EPI_GROUPS;
 constexpr int SEG_CAP = 1024;         // segments held in shared memory
 constexpr int NUM_ACC = 4;            // TMEM accumulators (4 x 128 columns = all of TMEM)
 constexpr int MAX_KP = 128;           // largest padded rank
 constexpr int NUM_YMAPS = 5;          // output boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
 constexpr int RING_PIECES = 32;       // pieces that may hold ring space at once
+// an accumulator slot and a ring barrier slot always serve the same epilogue group
+static_assert(NUM_ACC % EPI_GROUPS == 0 && RING_PIECES % EPI_GROUPS == 0, "slot ownership");
 
 struct SegEntry {
     int32_t row0;
@@ -74,7 +78,6 @@ struct Geometry {
     int32_t convert_x;  // x's dtype differs from the weights': round in shared memory
     int32_t n_tiles;    // ceil(N / BN)
     int32_t ring_rows, stages_w, stages_xo, stages_xr;
-    int32_t defer_release;   // release a piece's ring rows one piece later (ring holds >= 3 pieces)
     int32_t w_is_bf16;
     int32_t wmin;       // scheduling weight floor of a piece, in 8-row groups
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
@@ -265,11 +268,11 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         }
         for (int i = 0; i < NUM_ACC; ++i) {
             mbar_init(smem_u32(&acc_full[i]), 1);
-            mbar_init(smem_u32(&acc_empty[i]), EPI_WARPS);
+            mbar_init(smem_u32(&acc_empty[i]), 4);      // the four warps of one epilogue group
         }
         for (int i = 0; i < RING_PIECES; ++i) {
             mbar_init(smem_u32(&y_full[i]), 1);
-            mbar_init(smem_u32(&y_free[i]), EPI_WARPS);
+            mbar_init(smem_u32(&y_free[i]), 4);
         }
         fence_barrier_init();
     }
@@ -358,7 +361,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     const bool w_bf16 = geo.w_is_bf16 != 0;
     constexpr int CC = 128 / OUT_BYTES;              // columns per 128-byte chunk
     constexpr int NCH = BN / CC;                     // chunks per n-tile
-    constexpr int CPW = NCH / 2;                     // chunks per epilogue warp
+
     const int32_t RING_STRIDE = R * 128;             // bytes of one chunk's ring
 
     if (warp == 0) {
@@ -533,7 +536,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp % 4;                  // TMEM lane quadrant of this warp
-        const int half = (warp - EPI_WARP0) / 4; // which half of the chunks
+        const int grp = (warp - EPI_WARP0) / 4;  // this warp's group takes pieces t % EPI_GROUPS == grp
         const int r = q * 32 + lane;             // block row of this thread
         const int ri = r % GROUP;
         const bool out_bf16 = p.out_dt == SGMV_BF16;
@@ -542,10 +545,14 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         while (walk.next(pc)) {
             const int as = t % NUM_ACC;
             const int32_t pos = ring_place(head, (pc.rows + GROUP - 1) & ~(GROUP - 1), R);
+            if (t % EPI_GROUPS != grp) {   // the other group's piece
+                ++t;
+                continue;
+            }
             if (!warp_wait(smem_u32(&acc_full[as]), (t / NUM_ACC) & 1, abort_flag, DEVERR_TIMEOUT_EPILOGUE)) break;
             tc_fence_after();
-            // every warp waits, so that its release of this piece's ring rows below
-            // always lands in the right phase
+            // every warp of the group waits, so that its release of this piece's
+            // ring rows below always lands in the right phase
             if (!warp_wait(smem_u32(&y_full[t % RING_PIECES]), (t / RING_PIECES) & 1, abort_flag,
                            DEVERR_TIMEOUT_EPILOGUE))
                 break;
@@ -556,9 +563,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             const bool tail = r >= full_end;
             uint8_t* ring = smem + geo.off_y;
             const uint32_t taddr = tmem_base + (uint32_t)(as * BN) + ((uint32_t)(q * 32) << 16);
-#pragma unroll
-            for (int cc = 0; cc < CPW; ++cc) {
-                const int c = half * CPW + cc;
+#pragma unroll 1
+            for (int c = 0; c < NCH; ++c) {
                 if (c * CC >= ncols) break;     // warp-uniform
                 uint32_t v[CC];
 #pragma unroll
@@ -624,8 +630,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             if (lane == 0) {
                 const int32_t xcol0 = (int32_t)(p.off + pc.n0);
                 const int q_lo = q * 32, q_full = min(q * 32 + 32, full_end);
-                for (int cc = 0; cc < CPW; ++cc) {
-                    const int c = half * CPW + cc;
+                for (int c = 0; c < NCH; ++c) {
                     if (c * CC >= ncols) break;
                     for (int rr = q_lo; rr < q_full;) {
                         const int k = box_level(q_full - rr, 2);
@@ -635,15 +640,9 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     }
                 }
                 bulk_commit();
-                // release ring rows once the stores have read them: this piece's
-                // now, or (deep rings) the previous piece's, overlapping the drain
-                if (geo.defer_release) {
-                    bulk_wait_read<1>();
-                    if (t > 0) mbar_arrive(smem_u32(&y_free[(t - 1) % RING_PIECES]));
-                } else {
-                    bulk_wait_read<0>();
-                    mbar_arrive(smem_u32(&y_free[t % RING_PIECES]));
-                }
+                // release this piece's ring rows once the stores have read them
+                bulk_wait_read<0>();
+                mbar_arrive(smem_u32(&y_free[t % RING_PIECES]));
             }
             __syncwarp();
             ++t;
@@ -732,9 +731,6 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* 
             const int total = off + 1024;
             if (total > SMEM_OPTIN - SMEM_STATIC_RESERVE) continue;
             *total_out = total;
-            // A piece's rows may be released one piece late only if the ring can
-            // then still place the next piece: two pieces plus the skip at the wrap.
-            g.defer_release = rows >= 3 * BM;
             return true;
         }
     }

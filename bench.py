@@ -110,6 +110,24 @@ def recorded_traffic(workload, variant):
     return None
 
 
+# ---------------------------------------------------------------- ranks
+
+def reduce_over_ranks(total_ms, step_bytes, step_flops, tokens, device, world):
+    """Whole-job figures: the slowest rank's time, the sum of every rank's work.
+    Each rank runs its own batch (no data-path collective); this is the only
+    communication, outside the timed region."""
+    if world == 1:
+        return float(total_ms), float(step_bytes), float(step_flops), float(tokens)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    w = torch.tensor([float(step_bytes), float(step_flops), float(tokens)], dtype=torch.float64, device=device)
+    dist.all_reduce(w)
+    b, f, n = (float(v) for v in w.tolist())
+    return float(t.item()), b, f, n
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -273,19 +291,10 @@ def bench_ours(args, rank, world, device):
     del graphs
     assert sg.device_error(device) == 0, "a kernel reported a device-side error"
 
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
-
     step_bytes, step_flops, step_rows = step_accounting(p)
     call_bytes, _, _ = call_accounting(p, 0)
-    if world > 1:
-        tot = torch.tensor([step_bytes, step_flops, p.total_tokens], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(tot)
-        all_bytes, all_flops, all_tokens = [float(v) for v in tot.tolist()]
-    else:
-        all_bytes, all_flops, all_tokens = float(step_bytes), float(step_flops), float(p.total_tokens)
+    total_ms, all_bytes, all_flops, all_tokens = reduce_over_ranks(total_ms, step_bytes, step_flops,
+                                                                   p.total_tokens, device, world)
     ms_per_step = total_ms / K
     value = all_bytes * K / (total_ms * 1e-3) / 1e9
     avg_launch_ms = total_ms / (K * ncalls)
@@ -322,10 +331,7 @@ def bench_ours(args, rank, world, device):
             e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = reduce_over_ranks(e2e_ms, 0, 0, 0, device, world)[0]
         e2e = {"value": all_bytes * E / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / E, "steps": E}

@@ -110,6 +110,7 @@ struct Piece {
     int32_t blk_row0;     // row (of out and x) where the 128-row block starts
     int32_t rows;         // rows of the block (1 .. 128)
     int32_t n0;           // first column within the slice
+    int32_t shift;        // TMEM lane of the piece's first row (0, 32, 64 or 96)
     bool new_x;           // first piece of this x block in this CTA
     bool last_x;          // last piece of this x block in this CTA
 };
@@ -182,6 +183,10 @@ struct Walker {
         p.blk_row0 = s.row0 + rb * BM;
         p.rows = min(BM, s.rows - rb * BM);
         p.n0 = j * BN;
+        // A short block's n-tiles take turns in the TMEM lane quadrants, so that
+        // the epilogue warps of every quadrant share its work.
+        const int32_t nq = (p.rows + 31) / 32;
+        p.shift = nq == 1 ? 32 * (j % 4) : nq == 2 ? 64 * (j % 2) : 0;
         p.new_x = first || j == 0;
         first = false;
         cur += gcw;
@@ -516,7 +521,10 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             if (!warp_wait(smem_u32(&acc_empty[as]), ((t / NUM_ACC) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t a_base = smem_u32(smem + geo.off_xo + xs * geo.xo_bytes);
+                // A row m reads x row m - shift: the piece's rows land in TMEM lanes
+                // [shift, shift + rows); rows below come from unrelated shared memory
+                // and only fill lanes nobody reads.
+                const uint32_t a_base = smem_u32(smem + geo.off_xo + xs * geo.xo_bytes) - (uint32_t)(pc.shift * 16);
                 const uint32_t b_base = smem_u32(smem + geo.off_w + ws * geo.w_bytes);
                 const uint32_t d = tmem_base + (uint32_t)(as * BN);
 #pragma unroll
@@ -558,9 +566,10 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 break;
             const int full_end = pc.rows & ~(GROUP - 1);
             const int ncols = min(BN, (int)(p.N - pc.n0));
-            const bool valid = r < pc.rows;
+            const int pr = r - pc.shift;        // this thread's row within the piece
+            const bool valid = pr >= 0 && pr < pc.rows;
             // rows past the last whole group go straight to global memory from registers
-            const bool tail = r >= full_end;
+            const bool tail = pr >= full_end;
             uint8_t* ring = smem + geo.off_y;
             const uint32_t taddr = tmem_base + (uint32_t)(as * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
@@ -572,9 +581,9 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     tmem_ld32(taddr + (uint32_t)(c * CC + sub * 32), *reinterpret_cast<uint32_t(*)[32]>(v + sub * 32));
                 tmem_ld_wait();
                 if (valid) {
-                    uint8_t* rowp = ring + c * RING_STRIDE + (pos + r) * 128;
+                    uint8_t* rowp = ring + c * RING_STRIDE + (pos + pr) * 128;
                     uint4* grow = reinterpret_cast<uint4*>(reinterpret_cast<char*>(p.out) +
-                                                           ((int64_t)(pc.blk_row0 + r) * p.H + p.off + pc.n0 + c * CC) *
+                                                           ((int64_t)(pc.blk_row0 + pr) * p.H + p.off + pc.n0 + c * CC) *
                                                                OUT_BYTES);
                     const int kvalid = (min(CC, ncols - c * CC) * OUT_BYTES) / 16;   // 16-byte pieces in the slice
                     uint4 old[8];
@@ -629,7 +638,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             __syncwarp();
             if (lane == 0) {
                 const int32_t xcol0 = (int32_t)(p.off + pc.n0);
-                const int q_lo = q * 32, q_full = min(q * 32 + 32, full_end);
+                const int q_lo = max(q * 32 - pc.shift, 0), q_full = min(q * 32 + 32 - pc.shift, full_end);
                 for (int c = 0; c < NCH; ++c) {
                     if (c * CC >= ncols) break;
                     for (int rr = q_lo; rr < q_full;) {

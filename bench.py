@@ -204,6 +204,60 @@ def make_calls(p, dev_tensors, sg_abi, stream_handle_fn):
     return run, descs
 
 
+def make_multi_call(p, dev_tensors):
+    """Pre-marshalled arguments of ONE multi-slice call covering every slice."""
+    import segmented_gather_gemm_expand_b200 as sg
+    x, ws, y, meta = dev_tensors
+    xd, yd = sg._desc(x), sg._desc(y)
+    md = [sg._desc(t) for t in meta]
+    wd = [sg._desc(w) for w in ws]
+    n = len(wd)
+    arr = (ctypes.POINTER(sg._abi.SgmvTensor) * n)(*[ctypes.pointer(w) for w in wd])
+    offs = (ctypes.c_int64 * n)(*[c.slice_offset for c in p.calls])
+    keep = (xd, yd, md, wd, arr, offs)
+    lib = sg._lib
+
+    def run(stream):
+        rc = lib.sgmv_expand_multi_slice(ctypes.byref(xd), arr, n, ctypes.byref(yd),
+                                         *[ctypes.byref(t) for t in md], p.batches, p.max_seq_len, offs,
+                                         int(p.add_inputs), ctypes.c_void_p(stream))
+        if rc != 0:
+            raise sg.SgmvError(rc, "sgmv_expand_multi_slice")
+    run.keep = keep
+    return run
+
+
+def time_graph_region(step, steps, stream, torch):
+    """Capture `steps` calls of step(stream_handle) as graphs of <= STEPS_PER_GRAPH
+    steps, replay them once untimed, then time one replay of all of them with
+    CUDA events on `stream`.  Returns milliseconds."""
+    graphs = []
+    remaining = steps
+    while remaining > 0:
+        s = min(STEPS_PER_GRAPH, remaining)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            cs = torch.cuda.current_stream().cuda_stream
+            for _ in range(s):
+                step(cs)
+        graphs.append(g)
+        remaining -= s
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for g in graphs:
+            g.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    del graphs
+    return ms
+
+
 # ---------------------------------------------------------------- our arm
 
 def bench_ours(args, rank, world, device):
@@ -336,6 +390,28 @@ def bench_ours(args, rank, world, device):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / E, "steps": E}
 
+    # ---- the same step as ONE fused multi-slice launch (several slices only)
+    fused = None
+    if ncalls > 1 and not args.no_fused:
+        run_multi = make_multi_call(p, (x, ws, y, meta))
+        fv, fl = sg.plan_multi_slice(x, ws, y, *meta, p.batches, p.max_seq_len,
+                                     [c.slice_offset for c in p.calls], p.add_inputs)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                run_multi(stream.cuda_stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        fms = time_graph_region(run_multi, K, stream, torch)
+        fms = reduce_over_ranks(fms, 0, 0, 0, device, world)[0]
+        assert sg.device_error(device) == 0, "a kernel reported a device-side error"
+        f_ach = step_bytes / (fms / K * 1e-3) / 1e9
+        fused = {"entry_point": "sgmv_expand_multi_slice", "launches_per_step": fl,
+                 "variant": {1: "simt", 2: "tc"}.get(fv, "per-slice"),
+                 "ms_per_step": fms / K, "value": all_bytes * K / (fms * 1e-3) / 1e9, "unit": "GB/s",
+                 "achieved": f_ach, "frac": f_ach / peak, "bytes_per_launch": step_bytes / max(fl, 1),
+                 "note": "all slices of a step in one call; same bytes as the separate calls"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(p, budget_s=args.cpu_seconds)
@@ -368,6 +444,7 @@ def bench_ours(args, rank, world, device):
                      "launch_ms_note": "timed region / launches (back-to-back launches, gaps included)"},
         "gpu_launches": K * ncalls,
         "clocks": clocks,
+        "fused_multi_slice": fused,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "when": datetime.datetime.utcnow().isoformat() + "Z",
@@ -476,6 +553,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the extra timing of the step as one multi-slice call")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

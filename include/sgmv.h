@@ -88,6 +88,8 @@ enum {
     SGMV_ERR_STRIDE = -11,           /* a negative stride */
     SGMV_ERR_TOO_LARGE = -12,        /* sizes beyond the library's index range */
     SGMV_ERR_VARIANT = -13,          /* the forced kernel variant cannot run this call */
+    SGMV_ERR_NUM_SLICES = -14,       /* num_slices outside [1, SGMV_MAX_SLICES] */
+    SGMV_ERR_SLICE_OVERLAP = -15,    /* two non-empty slices of one call share a column */
     SGMV_ERR_CUDA = -20,             /* a CUDA runtime call failed */
     SGMV_ERR_LAUNCH = -21            /* a kernel launch failed */
 };
@@ -131,6 +133,50 @@ SGMV_API int sgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, con
               const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
               int64_t batches, int64_t max_seq_len, int64_t slice_offset, int64_t slice_size,
               int add_inputs, int* variant);
+
+/* Most slices one sgmv_expand_multi_slice call takes. */
+#define SGMV_MAX_SLICES 4
+
+/*
+ * sgmv_expand_multi_slice -- several slices of one fused output in one call:
+ * for each i < num_slices, the operation above with lora_b[i], slice_offset =
+ * slice_offsets[i] and slice_size = lora_b[i]'s N (its shape[-2]), all sharing
+ * inputs, out, the metadata and add_inputs.  The page explains that the
+ * expand-slice kernel is kept apart from plain sgmv_expand so that a later
+ * fused operator can update several slices in one launch ("Implementation:
+ * Predibase Lorax SGMV Expand Slice Kernel", Description), and that the
+ * slices are those of fused projections such as QKV or gate/up (Usage);
+ * this is that operator.
+ *
+ *   lora_b         array of num_slices descriptors, each as lora_b above; they
+ *                  may differ in N, strides and adapter count
+ *   num_slices     1 .. SGMV_MAX_SLICES
+ *   slice_offsets  HOST array of num_slices column offsets
+ *
+ * The slices' column ranges must be disjoint (else SGMV_ERR_SLICE_OVERLAP),
+ * so the result equals the num_slices single-slice calls in any order, bit
+ * for bit.  When the tensor-core kernel can take the whole set (same adapter
+ * count and weight dtype, the alignment rules it needs) it runs as ONE launch
+ * that shares the x tiles, the segment table and the prologue among the
+ * slices; otherwise each slice is launched on its own.  Every argument is
+ * validated before anything is enqueued.  Slices with N == 0 are skipped.
+ */
+SGMV_API int sgmv_expand_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const* lora_b, int num_slices,
+                            const sgmv_tensor* out, const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                            const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
+                            const int64_t* slice_offsets, int add_inputs, void* stream);
+
+/*
+ * sgmv_plan_multi_slice -- validate exactly as sgmv_expand_multi_slice does and
+ * report the variant (SGMV_VARIANT_TC when the slices run as one fused launch,
+ * SGMV_VARIANT_SIMT when the generic kernel is forced, 0 when nothing launches
+ * or the slices run as separate launches with their own variants) and, in
+ * *launches, how many kernel launches the call makes.  Launches nothing.
+ */
+SGMV_API int sgmv_plan_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const* lora_b, int num_slices,
+                          const sgmv_tensor* out, const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                          const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
+                          const int64_t* slice_offsets, int add_inputs, int* variant, int* launches);
 
 /*
  * sgmv_validate_metadata -- check the VALUES of the metadata on the device and

@@ -14,6 +14,10 @@ updates ``output_tensor[start_b + m, slice_offset:slice_offset + slice_size]``
 for every sequence b with ``lora_indices_tensor[b] != -1`` and token m, with
 ``inputs[start_b + m] @ lora_b_weights[idx_b].T`` (added to the old values when
 ``add_inputs``).
+
+``sgmv_expand_multi_slice`` updates several disjoint slices of one fused
+output (the QKV or gate/up projections the page's Usage section names) in a
+single call, which the page's Description anticipates as a fused operator.
 """
 import ctypes
 
@@ -21,7 +25,7 @@ import torch
 
 from . import _abi
 
-__all__ = ["sgmv_expand_slice", "plan", "validate_metadata", "set_variant", "device_error",
+__all__ = ["sgmv_expand_slice", "sgmv_expand_multi_slice", "plan", "plan_multi_slice", "validate_metadata", "set_variant", "device_error",
            "SgmvError", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "library_path"]
 
 VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC = _abi.VARIANT_AUTO, _abi.VARIANT_SIMT, _abi.VARIANT_TC
@@ -74,6 +78,61 @@ def sgmv_expand_slice(inputs, lora_b_weights, output_tensor, b_seq_start_loc, se
     if rc != 0:
         raise SgmvError(rc, "sgmv_expand_slice")
     return output_tensor
+
+
+def _multi_args(inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor,
+                lora_indices_tensor, slice_offsets):
+    lora_b_list = list(lora_b_list)
+    offs = [int(o) for o in slice_offsets]
+    if len(offs) != len(lora_b_list):
+        raise ValueError("slice_offsets must have one entry per lora_b tensor")
+    d = _args(inputs, output_tensor, output_tensor, b_seq_start_loc, seq_len_tensor,
+              lora_indices_tensor)
+    for w in lora_b_list:
+        if not w.is_cuda or w.device != output_tensor.device:
+            raise ValueError("all tensors must be CUDA tensors on the same device")
+    ws = [_desc(w) for w in lora_b_list]
+    n = len(ws)
+    arr = (ctypes.POINTER(_abi.SgmvTensor) * max(n, 1))(*[ctypes.pointer(w) for w in ws])
+    off_arr = (ctypes.c_int64 * max(n, 1))(*offs)
+    keep = (ws, arr, off_arr)   # the descriptors must outlive the call
+    return d[0], arr, n, d[2], d[3], d[4], d[5], off_arr, keep
+
+
+def sgmv_expand_multi_slice(inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor,
+                            lora_indices_tensor, batches, max_seq_length, slice_offsets,
+                            add_inputs=False):
+    """In-place expand-slice of every (lora_b_list[i], slice_offsets[i]) pair on
+    ``output_tensor`` in one call; slice i's size is ``lora_b_list[i].shape[-2]``.
+    The slices' column ranges must be disjoint."""
+    x, arr, n, out, s, l, idx, offs, _keep = _multi_args(
+        inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor,
+        slice_offsets)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_expand_multi_slice(ctypes.byref(x), arr, n, ctypes.byref(out), ctypes.byref(s),
+                                          ctypes.byref(l), ctypes.byref(idx), int(batches),
+                                          int(max_seq_length), offs, int(bool(add_inputs)),
+                                          _stream_handle(output_tensor.device))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_expand_multi_slice")
+    return output_tensor
+
+
+def plan_multi_slice(inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor,
+                     lora_indices_tensor, batches, max_seq_length, slice_offsets, add_inputs=False):
+    """(variant, launches) a multi-slice call with these arguments would make."""
+    x, arr, n, out, s, l, idx, offs, _keep = _multi_args(
+        inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor,
+        slice_offsets)
+    v, k = ctypes.c_int(0), ctypes.c_int(0)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_plan_multi_slice(ctypes.byref(x), arr, n, ctypes.byref(out), ctypes.byref(s),
+                                        ctypes.byref(l), ctypes.byref(idx), int(batches),
+                                        int(max_seq_length), offs, int(bool(add_inputs)),
+                                        ctypes.byref(v), ctypes.byref(k))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_plan_multi_slice")
+    return v.value, k.value
 
 
 def plan(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor,

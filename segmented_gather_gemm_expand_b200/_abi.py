@@ -20,8 +20,10 @@ STATUS_NAMES = {
     -4: "SGMV_ERR_RANK_MISMATCH", -5: "SGMV_ERR_SLICE_SIZE", -6: "SGMV_ERR_LAYOUT_4D",
     -7: "SGMV_ERR_OUT_NOT_CONTIGUOUS", -8: "SGMV_ERR_SLICE_RANGE", -9: "SGMV_ERR_BATCHES",
     -10: "SGMV_ERR_SHAPE", -11: "SGMV_ERR_STRIDE", -12: "SGMV_ERR_TOO_LARGE",
-    -13: "SGMV_ERR_VARIANT", -20: "SGMV_ERR_CUDA", -21: "SGMV_ERR_LAUNCH",
+    -13: "SGMV_ERR_VARIANT", -14: "SGMV_ERR_NUM_SLICES", -15: "SGMV_ERR_SLICE_OVERLAP",
+    -20: "SGMV_ERR_CUDA", -21: "SGMV_ERR_LAUNCH",
 }
+MAX_SLICES = 4
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
 
@@ -59,6 +61,13 @@ def load():
     lib.sgmv_expand_slice.argtypes = [P, P, P, P, P, P, i64, i64, i64, i64, i32, vp]
     lib.sgmv_plan.restype = i32
     lib.sgmv_plan.argtypes = [P, P, P, P, P, P, i64, i64, i64, i64, i32, ctypes.POINTER(i32)]
+    PP = ctypes.POINTER(P)
+    I64P = ctypes.POINTER(i64)
+    lib.sgmv_expand_multi_slice.restype = i32
+    lib.sgmv_expand_multi_slice.argtypes = [P, PP, i32, P, P, P, P, i64, i64, I64P, i32, vp]
+    lib.sgmv_plan_multi_slice.restype = i32
+    lib.sgmv_plan_multi_slice.argtypes = [P, PP, i32, P, P, P, P, i64, i64, I64P, i32,
+                                          ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.sgmv_validate_metadata.restype = i32
     lib.sgmv_validate_metadata.argtypes = [P, P, P, i64, i64, i64, vp, vp]
     lib.sgmv_status_string.restype = ctypes.c_char_p

@@ -27,6 +27,8 @@ __device__ void raise_device_error(int32_t bits) { atomicOr(&g_device_error, bit
 
 #include "tc_kernel.cuh"
 
+static_assert(SGMV_MAX_SLICES == sgmv::tc::MAX_SLICES, "one fused launch takes every slice of a call");
+
 using namespace sgmv;
 
 namespace {
@@ -185,10 +187,56 @@ int launch_simt(const Call& c, const DeviceInfo& dev, cudaStream_t stream) {
 
 // Which variant runs a validated, non-empty call.
 int choose_variant(const Call& c, const DeviceInfo& dev, int forced) {
-    const bool tc_ok = dev.cc_major == 10 && tc_supports(c.p);
+    const bool tc_ok = dev.cc_major == 10 && tc_supports(&c.p, 1);
     if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
     if (forced == SGMV_VARIANT_TC) return tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
     return tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
+}
+
+// Several slices of one output: validate each as a single call, then check
+// that the set is well formed (count, disjoint column ranges).  Fills the
+// non-empty slices into calls[0..*n_live).
+int validate_multi(const sgmv_tensor* x, const sgmv_tensor* const* ws, int num_slices, const sgmv_tensor* out,
+                   const sgmv_tensor* s, const sgmv_tensor* l, const sgmv_tensor* idx, int64_t batches,
+                   int64_t max_seq_len, const int64_t* offsets, int add_inputs, Call* calls, int* n_live) {
+    if (!ws || !offsets) return SGMV_ERR_NULL_ARG;
+    if (num_slices < 1 || num_slices > SGMV_MAX_SLICES) return SGMV_ERR_NUM_SLICES;
+    *n_live = 0;
+    int64_t lo[SGMV_MAX_SLICES], hi[SGMV_MAX_SLICES];
+    for (int i = 0; i < num_slices; ++i) {
+        if (!ws[i]) return SGMV_ERR_NULL_ARG;
+        const int64_t n = ws[i]->ndim >= 2 && ws[i]->ndim <= 4 ? ws[i]->shape[ws[i]->ndim - 2] : -1;
+        Call c;
+        const int rc = validate_call(x, ws[i], out, s, l, idx, batches, max_seq_len, offsets[i], n < 0 ? 0 : n,
+                                     add_inputs, &c);
+        if (rc) return rc;
+        lo[i] = offsets[i];
+        hi[i] = offsets[i] + c.p.N;
+        for (int j = 0; j < i; ++j)   // empty ranges overlap nothing
+            if (lo[i] < hi[i] && lo[j] < hi[j] && lo[i] < hi[j] && lo[j] < hi[i]) return SGMV_ERR_SLICE_OVERLAP;
+        if (!c.empty) calls[(*n_live)++] = c;
+    }
+    return SGMV_OK;
+}
+
+// How the live slices of a multi-slice call are launched: one fused
+// tensor-core launch, or (when that cannot take the set) one launch per
+// slice, each with its own variant.  Returns the fused variant or a status.
+int choose_multi(const Call* calls, int n, const DeviceInfo& dev, int forced, bool* fused) {
+    *fused = false;
+    if (forced != SGMV_VARIANT_SIMT && dev.cc_major == 10) {
+        Problem ps[SGMV_MAX_SLICES];
+        for (int i = 0; i < n; ++i) ps[i] = calls[i].p;
+        if (tc_supports(ps, n)) {
+            *fused = true;
+            return SGMV_VARIANT_TC;
+        }
+    }
+    for (int i = 0; i < n; ++i) {
+        const int v = choose_variant(calls[i], dev, forced);
+        if (v < 0) return v;
+    }
+    return forced == SGMV_VARIANT_SIMT ? (int)SGMV_VARIANT_SIMT : 0;
 }
 
 }  // namespace
@@ -209,7 +257,7 @@ int sgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, cons
     const int v = choose_variant(c, dev, g_forced_variant.load());
     if (v < 0) return v;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (v == SGMV_VARIANT_TC) return launch_tc(c.p, dev.sm_count, st);
+    if (v == SGMV_VARIANT_TC) return launch_tc(&c.p, 1, dev.sm_count, st);
     return launch_simt(c, dev, st);
 }
 
@@ -229,6 +277,59 @@ int sgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_t
     const int v = choose_variant(c, dev, g_forced_variant.load());
     if (v < 0) return v;
     *variant = v;
+    return SGMV_OK;
+}
+
+int sgmv_expand_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const* lora_b, int num_slices,
+                            const sgmv_tensor* out, const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                            const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
+                            const int64_t* slice_offsets, int add_inputs, void* stream) {
+    Call calls[SGMV_MAX_SLICES];
+    int n = 0;
+    int rc = validate_multi(inputs, lora_b, num_slices, out, seq_start, seq_len, lora_idx, batches, max_seq_len,
+                            slice_offsets, add_inputs, calls, &n);
+    if (rc) return rc;
+    if (n == 0) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    const int forced = g_forced_variant.load();
+    bool fused = false;
+    const int v = choose_multi(calls, n, dev, forced, &fused);
+    if (v < 0) return v;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (fused) {
+        Problem ps[SGMV_MAX_SLICES];
+        for (int i = 0; i < n; ++i) ps[i] = calls[i].p;
+        return launch_tc(ps, n, dev.sm_count, st);
+    }
+    for (int i = 0; i < n; ++i) {
+        const int vi = choose_variant(calls[i], dev, forced);
+        rc = vi == SGMV_VARIANT_TC ? launch_tc(&calls[i].p, 1, dev.sm_count, st) : launch_simt(calls[i], dev, st);
+        if (rc) return rc;
+    }
+    return SGMV_OK;
+}
+
+int sgmv_plan_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const* lora_b, int num_slices,
+                          const sgmv_tensor* out, const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                          const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
+                          const int64_t* slice_offsets, int add_inputs, int* variant, int* launches) {
+    if (!variant || !launches) return SGMV_ERR_NULL_ARG;
+    *variant = 0;
+    *launches = 0;
+    Call calls[SGMV_MAX_SLICES];
+    int n = 0;
+    int rc = validate_multi(inputs, lora_b, num_slices, out, seq_start, seq_len, lora_idx, batches, max_seq_len,
+                            slice_offsets, add_inputs, calls, &n);
+    if (rc) return rc;
+    if (n == 0) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    bool fused = false;
+    const int v = choose_multi(calls, n, dev, g_forced_variant.load(), &fused);
+    if (v < 0) return v;
+    *variant = v;
+    *launches = fused ? 1 : n;
     return SGMV_OK;
 }
 
@@ -275,6 +376,8 @@ const char* sgmv_status_string(int code) {
         case SGMV_ERR_STRIDE: return "negative stride";
         case SGMV_ERR_TOO_LARGE: return "sizes beyond the library's index range";
         case SGMV_ERR_VARIANT: return "the forced kernel variant cannot run this call";
+        case SGMV_ERR_NUM_SLICES: return "num_slices outside [1, SGMV_MAX_SLICES]";
+        case SGMV_ERR_SLICE_OVERLAP: return "two slices of a multi-slice call overlap";
         case SGMV_ERR_CUDA: return "a CUDA runtime call failed";
         case SGMV_ERR_LAUNCH: return "kernel launch failed";
         default: return "unknown status";

@@ -5,11 +5,12 @@
 
 namespace sgmv {
 
-// True when the tensor-core kernel can run this call (dtypes, rank,
-// alignment, sizes); otherwise the generic kernel runs it.
-bool tc_supports(const Problem& p);
+// True when the tensor-core kernel can run these `nsl` slices of one output
+// (dtypes, rank, alignment, sizes) in one launch; otherwise the generic kernel
+// runs them, one launch per slice.
+bool tc_supports(const Problem* slices, int nsl);
 
-// Enqueue the tensor-core kernel.  Returns an SGMV status.
-int launch_tc(const Problem& p, int sm_count, cudaStream_t stream);
+// Enqueue the tensor-core kernel for `nsl` slices.  Returns an SGMV status.
+int launch_tc(const Problem* slices, int nsl, int sm_count, cudaStream_t stream);
 
 }  // namespace sgmv

@@ -59,6 +59,7 @@ constexpr int NUM_ACC = 4;            // TMEM accumulators (4 x 128 columns = al
 constexpr int MAX_KP = 128;           // largest padded rank
 constexpr int NUM_YMAPS = 5;          // output boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
+constexpr int MAX_SLICES = 4;         // slices of one output updated by one launch
 constexpr int RING_PIECES = 32;       // pieces that may hold ring space at once
 // an accumulator slot and a ring barrier slot always serve the same epilogue group
 static_assert(NUM_ACC % EPI_GROUPS == 0 && RING_PIECES % EPI_GROUPS == 0, "slot ownership");
@@ -76,7 +77,7 @@ struct Geometry {
     int32_t Kp;         // rank padded to a multiple of 16
     int32_t x_bytes;    // element size of x
     int32_t convert_x;  // x's dtype differs from the weights': round in shared memory
-    int32_t n_tiles;    // ceil(N / BN)
+    int32_t n_tiles;    // n-tiles of all slices together
     int32_t ring_rows, stages_w, stages_xo, stages_xr;
     int32_t w_is_bf16;
     int32_t wmin;       // scheduling weight floor of a piece, in 8-row groups
@@ -96,11 +97,21 @@ struct Geometry {
 };
 
 struct YMaps {
-    CUtensorMap m[NUM_YMAPS];
+    CUtensorMap m[MAX_SLICES][NUM_YMAPS];
 };
 
 struct WMaps {
-    CUtensorMap m[MAX_WBLK];
+    CUtensorMap m[MAX_SLICES][MAX_WBLK];
+};
+
+// The slices of one launch: slice s covers output columns [off[s], off[s] + N[s])
+// with its own B; its n-tiles are numbers [tile0[s], tile0[s + 1]) of a piece's
+// row block.
+struct Slices {
+    int32_t count;
+    int32_t tile0[MAX_SLICES + 1];
+    int64_t off[MAX_SLICES];
+    int64_t N[MAX_SLICES];
 };
 
 // ---------------------------------------------------------------- scheduler
@@ -110,6 +121,7 @@ struct Piece {
     int32_t blk_row0;     // row (of out and x) where the 128-row block starts
     int32_t rows;         // rows of the block (1 .. 128)
     int32_t n0;           // first column within the slice
+    int32_t slice;
     int32_t shift;        // TMEM lane of the piece's first row (0, 32, 64 or 96)
     bool new_x;           // first piece of this x block in this CTA
     bool last_x;          // last piece of this x block in this CTA
@@ -119,6 +131,7 @@ struct Piece {
 // Every role runs an identical copy, so all roles see the same sequence.
 struct Walker {
     const SegEntry* segs;
+    const int32_t* tile0;   // first n-tile of each slice
     int32_t nseg, n_tiles, wmin;
     int32_t i, rb, j;     // segment, row block, n-tile
     int32_t G, nblk, gcw; // groups and blocks of segment i; weight of a piece of block rb
@@ -182,7 +195,10 @@ struct Walker {
         p.adapter = s.adapter;
         p.blk_row0 = s.row0 + rb * BM;
         p.rows = min(BM, s.rows - rb * BM);
-        p.n0 = j * BN;
+        int32_t sl = 0;
+        while (j >= tile0[sl + 1]) ++sl;
+        p.slice = sl;
+        p.n0 = (j - tile0[sl]) * BN;
         // A short block's n-tiles take turns in the TMEM lane quadrants, so that
         // the epilogue warps of every quadrant share its work.
         const int32_t nq = (p.rows + 31) / 32;
@@ -229,7 +245,8 @@ __device__ __forceinline__ int32_t ring_place(int32_t& head, int32_t rows8, int3
 template <int OUT_BYTES, bool ADD>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constant__ CUtensorMap tmap_x,
-                       const __grid_constant__ YMaps ymaps, Problem p, Geometry geo) {
+                       const __grid_constant__ YMaps ymaps, Problem p, Geometry geo,
+                       const __grid_constant__ Slices sl) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -282,9 +299,11 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        for (int b = 0; b < geo.w_nblk; ++b) prefetch_tmap(&wmaps.m[b]);
         prefetch_tmap(&tmap_x);
-        for (int k = 0; k < NUM_YMAPS; ++k) prefetch_tmap(&ymaps.m[k]);
+        for (int i = 0; i < sl.count; ++i) {
+            for (int b = 0; b < geo.w_nblk; ++b) prefetch_tmap(&wmaps.m[i][b]);
+            for (int k = 0; k < NUM_YMAPS; ++k) prefetch_tmap(&ymaps.m[i][k]);
+        }
     }
     if (warp == 1) tmem_alloc(smem_u32(&s_tmem_base), NUM_ACC * BN);
 
@@ -357,6 +376,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     const int32_t U = s_total_units;
     Walker walk;
     walk.segs = segs;
+    walk.tile0 = sl.tile0;
     walk.nseg = nseg;
     walk.n_tiles = geo.n_tiles;
     walk.wmin = geo.wmin;
@@ -405,7 +425,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                         break;
                     mbar_expect_tx(smem_u32(&w_full[s]), w_bytes);
                     for (int b = 0; b < geo.w_nblk; ++b)
-                        tma_load_3d(smem_u32(smem + geo.off_w + s * geo.w_bytes + geo.w_blk_off[b]), &wmaps.m[b],
+                        tma_load_3d(smem_u32(smem + geo.off_w + s * geo.w_bytes + geo.w_blk_off[b]), &wmaps.m[pc.slice][b],
                                     geo.w_blk_k0[b], pc.n0, pc.adapter, smem_u32(&w_full[s]), pol_keep);
                 }
                 ++t;
@@ -439,15 +459,15 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 ends[t % RING_PIECES] = head;
                 const uint32_t bar = smem_u32(&y_full[t % RING_PIECES]);
                 if (ADD) {
-                    const int ncols = min(BN, (int)(p.N - pc.n0));
+                    const int ncols = min(BN, (int)(sl.N[pc.slice] - pc.n0));
                     const int nch = (ncols + CC - 1) / CC;
                     mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
                     const uint32_t ring = smem_u32(smem + geo.off_y);
-                    const int32_t xcol0 = (int32_t)(p.off + pc.n0);
+                    const int32_t xcol0 = (int32_t)(sl.off[pc.slice] + pc.n0);
                     for (int c = 0; c < nch; ++c) {
                         for (int r = 0; r < rows8;) {
                             const int k = box_level(rows8 - r, NUM_YMAPS - 1);
-                            tma_load_2d(ring + c * RING_STRIDE + (pos + r) * 128, &ymaps.m[k], xcol0 + c * CC,
+                            tma_load_2d(ring + c * RING_STRIDE + (pos + r) * 128, &ymaps.m[pc.slice][k], xcol0 + c * CC,
                                         pc.blk_row0 + r, bar, pol_stream);
                             r += GROUP << k;
                         }
@@ -565,7 +585,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                            DEVERR_TIMEOUT_EPILOGUE))
                 break;
             const int full_end = pc.rows & ~(GROUP - 1);
-            const int ncols = min(BN, (int)(p.N - pc.n0));
+            const int ncols = min(BN, (int)(sl.N[pc.slice] - pc.n0));
+            const int64_t col0 = sl.off[pc.slice] + pc.n0;   // first output column of the piece
             const int pr = r - pc.shift;        // this thread's row within the piece
             const bool valid = pr >= 0 && pr < pc.rows;
             // rows past the last whole group go straight to global memory from registers
@@ -583,7 +604,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 if (valid) {
                     uint8_t* rowp = ring + c * RING_STRIDE + (pos + pr) * 128;
                     uint4* grow = reinterpret_cast<uint4*>(reinterpret_cast<char*>(p.out) +
-                                                           ((int64_t)(pc.blk_row0 + pr) * p.H + p.off + pc.n0 + c * CC) *
+                                                           ((int64_t)(pc.blk_row0 + pr) * p.H + col0 + c * CC) *
                                                                OUT_BYTES);
                     const int kvalid = (min(CC, ncols - c * CC) * OUT_BYTES) / 16;   // 16-byte pieces in the slice
                     uint4 old[8];
@@ -637,13 +658,13 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                const int32_t xcol0 = (int32_t)(p.off + pc.n0);
+                const int32_t xcol0 = (int32_t)col0;
                 const int q_lo = max(q * 32 - pc.shift, 0), q_full = min(q * 32 + 32 - pc.shift, full_end);
                 for (int c = 0; c < NCH; ++c) {
                     if (c * CC >= ncols) break;
                     for (int rr = q_lo; rr < q_full;) {
                         const int k = box_level(q_full - rr, 2);
-                        tma_store_2d(&ymaps.m[k], xcol0 + c * CC, pc.blk_row0 + rr,
+                        tma_store_2d(&ymaps.m[pc.slice][k], xcol0 + c * CC, pc.blk_row0 + rr,
                                      smem_u32(ring + c * RING_STRIDE + (pos + rr) * 128));
                         rr += GROUP << k;
                     }
@@ -699,6 +720,7 @@ struct Plan {
     WMaps tw;
     CUtensorMap tx;
     YMaps ty;
+    Slices sl;
 };
 
 // Scheduling weight floor of a piece (8-row groups): a piece of a few rows
@@ -746,8 +768,8 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* 
     return false;
 }
 
-// Everything the tensor-core kernel needs, or false if it cannot take the call.
-inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
+// Conditions one slice must meet for the tensor-core kernel.
+inline bool slice_ok(const Problem& p) {
     const int64_t sx = elem_bytes(p.x_dt), so = elem_bytes(p.out_dt);
     if (p.K < 8 || p.K > MAX_KP || p.K % 8 != 0) return false;
     if (p.x_cs != 1 || p.w_ks != 1) return false;
@@ -760,7 +782,34 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
     if (p.out_rows >= (int64_t(1) << 31) || p.x_rows >= (int64_t(1) << 31) || p.off + p.N >= (int64_t(1) << 32))
         return false;
     if (p.lora_num >= (int64_t(1) << 31)) return false;
-    const int64_t n_tiles = (p.N + BN - 1) / BN;
+    return true;
+}
+
+// Everything the tensor-core kernel needs for `nsl` slices of one output
+// (sharing x, the metadata and the adapter count), or false if it cannot
+// take the call.
+inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
+    if (nsl < 1 || nsl > MAX_SLICES) return false;
+    const Problem& p = ps[0];
+    for (int i = 0; i < nsl; ++i) {
+        if (!slice_ok(ps[i]) || ps[i].w_dt != p.w_dt || ps[i].lora_num != p.lora_num) return false;
+        if (ps[i].N == 0) return false;
+    }
+    const int64_t sx = elem_bytes(p.x_dt), so = elem_bytes(p.out_dt);
+    Slices& sl = out->sl;
+    sl.count = nsl;
+    sl.tile0[0] = 0;
+    for (int i = 0; i < nsl; ++i) {
+        sl.off[i] = ps[i].off;
+        sl.N[i] = ps[i].N;
+        sl.tile0[i + 1] = sl.tile0[i] + (int32_t)((ps[i].N + BN - 1) / BN);
+    }
+    for (int i = nsl; i < MAX_SLICES; ++i) {
+        sl.off[i] = 0;
+        sl.N[i] = 0;
+        sl.tile0[i + 1] = sl.tile0[i];
+    }
+    const int64_t n_tiles = sl.tile0[nsl];
     const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int64_t max_pieces = (t_lim / BM + p.batches + 1) * n_tiles;
     const int64_t weight_bound = (t_lim / GROUP + p.batches + 1) * n_tiles + PIECE_WEIGHT_FLOOR * max_pieces;
@@ -824,7 +873,9 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
     if (!enc) return false;
     const cuuint32_t ones[5] = {1, 1, 1, 1, 1};
     // B: (K, N rows, adapters); one box per K block, rows of 2*kb bytes swizzled by their width
+    for (int si = 0; si < nsl; ++si)
     for (int b = 0; b < g.w_nblk; ++b) {
+        const Problem& p = ps[si];
         const cuuint64_t dims[3] = {(cuuint64_t)p.K, (cuuint64_t)p.N, (cuuint64_t)p.lora_num};
         cuuint64_t a_stride = (cuuint64_t)(p.w_as * 2);
         if (p.lora_num == 1) a_stride = (cuuint64_t)round_up((int32_t)(p.N * p.w_ns * 2), 16);
@@ -835,7 +886,7 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
                                       : kb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                       : kb == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                  : CU_TENSOR_MAP_SWIZZLE_NONE;
-        if (enc(&out->tw.m[b], CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(p.w), dims, strides, box, ones,
+        if (enc(&out->tw.m[si][b], CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(p.w), dims, strides, box, ones,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
@@ -862,12 +913,14 @@ inline bool make_plan(const Problem& p, int sm_count, Plan* out) {
     }
     // out: columns [0, off + N) of each row (clipping at the slice end); boxes of
     // 8 << k rows x 128 bytes with the 128-byte swizzle
+    for (int si = 0; si < nsl; ++si)
     for (int k = 0; k < NUM_YMAPS; ++k) {
+        const Problem& p = ps[si];
         const cuuint64_t dims[2] = {(cuuint64_t)(p.off + p.N), (cuuint64_t)p.out_rows};
         const cuuint64_t strides[1] = {(cuuint64_t)(p.H * so)};
         const cuuint32_t box[2] = {(cuuint32_t)(128 / so), (cuuint32_t)(GROUP << k)};
         const CUtensorMapDataType dt = so == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-        if (enc(&out->ty.m[k], dt, 2, p.out, dims, strides, box, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        if (enc(&out->ty.m[si][k], dt, 2, p.out, dims, strides, box, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
@@ -898,20 +951,21 @@ int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, pl.tw, pl.tx, pl.ty, p, pl.geo) != cudaSuccess) return SGMV_ERR_LAUNCH;
+    if (cudaLaunchKernelEx(&cfg, kern, pl.tw, pl.tx, pl.ty, p, pl.geo, pl.sl) != cudaSuccess) return SGMV_ERR_LAUNCH;
     return SGMV_OK;
 }
 
 }  // namespace tc
 
-bool tc_supports(const Problem& p) {
+bool tc_supports(const Problem* ps, int nsl) {
     tc::Plan pl;
-    return tc::make_plan(p, 148, &pl);
+    return tc::make_plan(ps, nsl, 148, &pl);
 }
 
-int launch_tc(const Problem& p, int sm_count, cudaStream_t stream) {
+int launch_tc(const Problem* ps, int nsl, int sm_count, cudaStream_t stream) {
     tc::Plan pl;
-    if (!tc::make_plan(p, sm_count, &pl)) return SGMV_ERR_VARIANT;
+    if (!tc::make_plan(ps, nsl, sm_count, &pl)) return SGMV_ERR_VARIANT;
+    const Problem& p = ps[0];
     if (tc::elem_bytes(p.out_dt) == 4) {
         return p.add ? tc::launch_instance<4, true>(pl, p, stream) : tc::launch_instance<4, false>(pl, p, stream);
     }

@@ -133,3 +133,17 @@ def compare(gpu: np.ndarray, ref: np.ndarray, y0: np.ndarray, p: gen.Problem, ro
     assert np.all(err <= tol), (f"max err {err.max():.3g} over tol; worst gpu={g[finite][worst]!r} "
                                 f"ref={r[finite][worst]!r} tol={tol[worst]:.3g}")
     return float(err.max()) if err.size else 0.0
+
+
+def run_multi(dp: DeviceProblem, calls=None, out=None, plan_only=False):
+    """All (or the listed) slice calls of dp's problem as ONE multi-slice call.
+
+    plan_only: return (variant, launches) instead of running."""
+    import segmented_gather_gemm_expand_b200 as sg
+    p = dp.p
+    calls = list(range(len(p.calls))) if calls is None else list(calls)
+    ws = [dp.ws[c] for c in calls]
+    offs = [p.calls[c].slice_offset for c in calls]
+    y = dp.y if out is None else out
+    fn = sg.plan_multi_slice if plan_only else sg.sgmv_expand_multi_slice
+    return fn(dp.x, ws, y, dp.start, dp.len, dp.idx, p.batches, p.max_seq_len, offs, p.add_inputs)

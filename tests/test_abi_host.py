@@ -147,3 +147,75 @@ def test_empty_calls_need_no_device_and_launch_nothing():
     assert call(good_args(batches=0)) == 0
     empty_w = _abi.make_tensor(FAKE, _abi.BF16, (A, 0, K), (0, K, 1))
     assert call(good_args(w=empty_w, size=0)) == 0
+
+
+# --- several slices of one output (sgmv_expand_multi_slice) -----------------
+
+def call_multi(a, ws, offs, n=None):
+    lib = _abi.load()
+    r = ctypes.byref
+    n = len(ws) if n is None else n
+    arr = (ctypes.POINTER(_abi.SgmvTensor) * max(len(ws), 1))(*[ctypes.pointer(w) for w in ws])
+    off_arr = (ctypes.c_int64 * max(len(offs), 1))(*offs)
+    rc = lib.sgmv_expand_multi_slice(r(a["x"]), arr, n, r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]),
+                                     a["batches"], a["max_seq_len"], off_arr, a["add"], None)
+    v, k = ctypes.c_int(-1), ctypes.c_int(-1)
+    rc2 = lib.sgmv_plan_multi_slice(r(a["x"]), arr, n, r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]),
+                                    a["batches"], a["max_seq_len"], off_arr, a["add"], r(v), r(k))
+    assert rc2 == rc
+    if rc:
+        assert v.value == 0 and k.value == 0
+    return rc
+
+
+def wslice(n):
+    return _abi.make_tensor(FAKE, _abi.BF16, (A, n, K), (n * K, K, 1))
+
+
+def test_multi_slice_overlapping_ranges_rejected():
+    a = good_args()
+    assert call_multi(a, [wslice(128), wslice(128)], [0, 64]) == _abi.STATUS["SGMV_ERR_SLICE_OVERLAP"]
+    assert call_multi(a, [wslice(128), wslice(64), wslice(64)], [0, 256, 300]) == \
+        _abi.STATUS["SGMV_ERR_SLICE_OVERLAP"]
+    # the same slice twice
+    assert call_multi(a, [wslice(128), wslice(128)], [128, 128]) == _abi.STATUS["SGMV_ERR_SLICE_OVERLAP"]
+
+
+def test_multi_slice_count_and_null_checks():
+    lib = _abi.load()
+    a = good_args()
+    assert call_multi(a, [wslice(64)] * 5, [0, 64, 128, 192, 256]) == _abi.STATUS["SGMV_ERR_NUM_SLICES"]
+    assert call_multi(a, [wslice(64)], [0], n=0) == _abi.STATUS["SGMV_ERR_NUM_SLICES"]
+    r = ctypes.byref
+    off_arr = (ctypes.c_int64 * 1)(0)
+    assert lib.sgmv_expand_multi_slice(r(a["x"]), None, 1, r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]),
+                                       4, 7, off_arr, 0, None) == _abi.STATUS["SGMV_ERR_NULL_ARG"]
+    arr = (ctypes.POINTER(_abi.SgmvTensor) * 1)(ctypes.pointer(wslice(64)))
+    assert lib.sgmv_expand_multi_slice(r(a["x"]), arr, 1, r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]),
+                                       4, 7, None, 0, None) == _abi.STATUS["SGMV_ERR_NULL_ARG"]
+    arr2 = (ctypes.POINTER(_abi.SgmvTensor) * 2)(ctypes.pointer(wslice(64)), None)
+    off2 = (ctypes.c_int64 * 2)(0, 64)
+    assert lib.sgmv_expand_multi_slice(r(a["x"]), arr2, 2, r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]),
+                                       4, 7, off2, 0, None) == _abi.STATUS["SGMV_ERR_NULL_ARG"]
+
+
+def test_multi_slice_validates_every_slice():
+    a = good_args()
+    # slice 2 reaches past the output width
+    assert call_multi(a, [wslice(128), wslice(128)], [0, 300]) == _abi.STATUS["SGMV_ERR_SLICE_RANGE"]
+    # slice 2 has the wrong rank
+    bad_rank = _abi.make_tensor(FAKE, _abi.BF16, (A, 64, 8), (64 * 8, 8, 1))
+    assert call_multi(a, [wslice(64), bad_rank], [0, 64]) == _abi.STATUS["SGMV_ERR_RANK_MISMATCH"]
+    bad_dt = _abi.make_tensor(FAKE, _abi.F32, (A, 64, K), (64 * K, K, 1))
+    assert call_multi(a, [bad_dt], [0]) == _abi.STATUS["SGMV_ERR_DTYPE"]
+    assert call_multi(a, [wslice(64), _abi.make_tensor(FAKE, _abi.BF16, (64, K), (K, 1))], [0, 64]) == \
+        _abi.STATUS["SGMV_ERR_NDIM"]
+
+
+def test_multi_slice_empty_needs_no_device():
+    # every slice empty, or no batches: OK before any CUDA call
+    a = good_args()
+    assert call_multi(a, [wslice(0), wslice(0)], [0, 0]) == 0
+    assert call_multi(good_args(batches=0), [wslice(128), wslice(128)], [0, 128]) == 0
+    # an empty slice inside a non-empty one overlaps nothing
+    assert call_multi(good_args(batches=0), [wslice(128), wslice(0)], [0, 64]) == 0

@@ -53,7 +53,7 @@ def load():
         return _lib
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libsgmv.so not found at {LIB_PATH}; build it with "
-                          "`python -m segmented_gather_gemm_expand_b200.build`")
+                          "`python segmented_gather_gemm_expand_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER(SgmvTensor)
     i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p

@@ -1,6 +1,7 @@
 """Build libsgmv.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-Usage: python -m segmented_gather_gemm_expand_b200.build [--force]
+Usage: python segmented_gather_gemm_expand_b200/build.py [--force]
+(run as a script: importing the package needs the library this builds)
 """
 import glob
 import os

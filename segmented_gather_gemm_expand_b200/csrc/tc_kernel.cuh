@@ -29,8 +29,9 @@
 // segment, 128-column n-tile); pieces are ordered with the n-tile fastest, so
 // the x block is staged once and reused across every n-tile.  Every CTA builds
 // the table of segments in shared memory (the guards of sgmv.h applied),
-// weighs each piece as max(its 8-row groups, a floor for the fixed per-piece
-// cost), and takes the pieces that start in its equal share of the weight.
+// weighs each piece as its 8-row groups plus a fixed part (its B tile and the
+// per-piece pipeline work), and takes the pieces that start in its equal share
+// of the total weight.
 // Every wait on an mbarrier is bounded; a wait that gives up sets the device
 // error word and makes the CTA leave its loops.
 #pragma once
@@ -80,7 +81,8 @@ struct Geometry {
     int32_t n_tiles;    // n-tiles of all slices together
     int32_t ring_rows, stages_w, stages_xo, stages_xr;
     int32_t w_is_bf16;
-    int32_t wmin;       // scheduling weight floor of a piece, in 8-row groups
+    int32_t wmin, wfix; // scheduling weight of a piece: max(its 8-row groups, wmin) + wfix
+    int32_t rr;         // 1: the kernel may hand out pieces round-robin (see the segment table)
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
     // (rows of 2*kb bytes, swizzled by the row width) at w_blk_off in a stage
     int32_t w_nblk;
@@ -91,6 +93,7 @@ struct Geometry {
     int32_t ksteps;
     uint64_t b_desc_rel[MAX_KP / 16];
     uint32_t b_off[MAX_KP / 16];
+
     // shared memory offsets (bytes, from the 1024-aligned base)
     int32_t off_y, off_w, off_xo, off_xr, off_seg, off_ends, off_bar;
     int32_t w_bytes, xo_bytes, xr_bytes;
@@ -104,6 +107,8 @@ struct WMaps {
     CUtensorMap m[MAX_SLICES][MAX_WBLK];
 };
 
+
+
 // The slices of one launch: slice s covers output columns [off[s], off[s] + N[s])
 // with its own B; its n-tiles are numbers [tile0[s], tile0[s + 1]) of a piece's
 // row block.
@@ -114,6 +119,15 @@ struct Slices {
     int64_t N[MAX_SLICES];
 };
 
+// The slice table as the kernel reads it, copied into shared memory at the
+// start: reading it from the parameter space through a pointer with a
+// data-dependent index costs a slow generic load on every piece.
+struct SliceTable {
+    int32_t tile0[MAX_SLICES + 1];
+    int32_t off[MAX_SLICES];
+    int32_t N[MAX_SLICES];
+};
+
 // ---------------------------------------------------------------- scheduler
 
 struct Piece {
@@ -121,28 +135,37 @@ struct Piece {
     int32_t blk_row0;     // row (of out and x) where the 128-row block starts
     int32_t rows;         // rows of the block (1 .. 128)
     int32_t n0;           // first column within the slice
+    int32_t col0;         // first output column of the piece
+    int32_t ncols;        // columns of the piece (1 .. BN)
     int32_t slice;
     int32_t shift;        // TMEM lane of the piece's first row (0, 32, 64 or 96)
+    int32_t t;            // index of the piece among this CTA's pieces
     bool new_x;           // first piece of this x block in this CTA
     bool last_x;          // last piece of this x block in this CTA
 };
 
-// Walks the pieces whose start weight lies in the CTA's range [w0, w_end).
+// Walks the CTA's pieces in one of two ways:
+//   - contiguous: the pieces whose start weight lies in [w0, w_end) (seek);
+//   - round-robin: pieces c, c + stride, c + 2*stride, ... of the sequence of all
+//     pieces (seek_rr), so that every CTA gets the same mix of long and short
+//     pieces and, at any moment, the CTAs together cover whole output rows.
 // Every role runs an identical copy, so all roles see the same sequence.
 struct Walker {
     const SegEntry* segs;
-    const int32_t* tile0;   // first n-tile of each slice
-    int32_t nseg, n_tiles, wmin;
+    const SliceTable* st;   // shared memory
+    int32_t nseg, n_tiles, wmin, wfix;
     int32_t i, rb, j;     // segment, row block, n-tile
+    int32_t t;            // pieces handed out so far
     int32_t G, nblk, gcw; // groups and blocks of segment i; weight of a piece of block rb
     int32_t cur, w_end;   // start weight of the next piece; end of the range
+    int32_t stride;       // round-robin stride (0: contiguous)
     bool first;
 
     __device__ void load_segment_geometry() {
         G = (segs[i].rows + GROUP - 1) / GROUP;
         nblk = (G + GROUPS_PER_BLOCK - 1) / GROUPS_PER_BLOCK;
     }
-    __device__ void set_block() { gcw = max(min(GROUPS_PER_BLOCK, G - rb * GROUPS_PER_BLOCK), wmin); }
+    __device__ void set_block() { gcw = max(min(GROUPS_PER_BLOCK, G - rb * GROUPS_PER_BLOCK), wmin) + wfix; }
     __device__ void skip_empty() {
         while (i < nseg && segs[i].rows == 0) ++i;
         if (i < nseg) {
@@ -153,7 +176,9 @@ struct Walker {
 
     __device__ void seek(int32_t w0, int32_t w1) {
         w_end = w1;
+        stride = 0;
         first = true;
+        t = 0;
         i = nseg;
         rb = j = 0;
         cur = w1;
@@ -168,7 +193,7 @@ struct Walker {
         skip_empty();
         if (i >= nseg) return;
         const int32_t local = w0 - segs[i].prefix;
-        const int32_t bw = max(GROUPS_PER_BLOCK, wmin) * n_tiles;   // weight of a full row block
+        const int32_t bw = (max(GROUPS_PER_BLOCK, wmin) + wfix) * n_tiles;   // weight of a full row block
         rb = min(local / bw, nblk - 1);
         set_block();
         const int32_t rem = local - rb * bw;
@@ -189,20 +214,78 @@ struct Walker {
         cur = segs[i].prefix + rb * bw + j * gcw;
     }
 
-    __device__ bool next(Piece& p) {
-        if (i >= nseg || cur >= w_end) return false;
+    // Round-robin: the segment table's prefixes count pieces.  Moves to piece
+    // `local` of segment i (or of a later segment), skipping empty ones.
+    __device__ void advance_rr(int32_t local) {
+        while (i < nseg && local >= nblk * n_tiles) {
+            local -= nblk * n_tiles;
+            ++i;
+            while (i < nseg && segs[i].rows == 0) ++i;
+            if (i < nseg) load_segment_geometry();
+        }
+        rb = local / n_tiles;
+        j = local - rb * n_tiles;
+    }
+
+    __device__ void seek_rr(int32_t c, int32_t step) {
+        stride = step;
+        first = true;
+        t = 0;
+        i = nseg;
+        rb = j = 0;
+        if (nseg == 0) return;
+        int lo = 0, hi = nseg - 1;   // last segment whose prefix <= c
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (segs[mid].prefix <= c) lo = mid;
+            else hi = mid - 1;
+        }
+        i = lo;
+        while (i < nseg && segs[i].rows == 0) ++i;
+        if (i >= nseg) return;
+        load_segment_geometry();
+        advance_rr(c - segs[i].prefix);
+    }
+
+    __device__ bool next_rr(Piece& p) {
+        if (i >= nseg) return false;
+        const int32_t pi = i, prb = rb;
+        fill(p);
+        p.new_x = first || i != last_i || rb != last_rb;
+        first = false;
+        last_i = i;
+        last_rb = rb;
+        advance_rr(rb * n_tiles + j + stride);
+        p.last_x = i >= nseg || i != pi || rb != prb;
+        return true;
+    }
+    int32_t last_i, last_rb;
+
+    // The piece at (i, rb, j), and the quadrant turn of the t-th piece.
+    __device__ void fill(Piece& p) {
         const SegEntry s = segs[i];
         p.adapter = s.adapter;
         p.blk_row0 = s.row0 + rb * BM;
         p.rows = min(BM, s.rows - rb * BM);
         int32_t sl = 0;
-        while (j >= tile0[sl + 1]) ++sl;
+        while (j >= st->tile0[sl + 1]) ++sl;
         p.slice = sl;
-        p.n0 = (j - tile0[sl]) * BN;
-        // A short block's n-tiles take turns in the TMEM lane quadrants, so that
-        // the epilogue warps of every quadrant share its work.
+        p.n0 = (j - st->tile0[sl]) * BN;
+        p.col0 = st->off[sl] + p.n0;
+        p.ncols = min(BN, st->N[sl] - p.n0);
+        // Short pieces take turns in the TMEM lane quadrants, so that the
+        // epilogue warps of every quadrant share them: the pieces of one
+        // epilogue group (every EPI_GROUPS-th) cycle through the quadrants.
         const int32_t nq = (p.rows + 31) / 32;
-        p.shift = nq == 1 ? 32 * (j % 4) : nq == 2 ? 64 * (j % 2) : 0;
+        const int32_t turn = t / EPI_GROUPS;
+        p.shift = nq == 1 ? 32 * (turn % 4) : nq == 2 ? 64 * (turn % 2) : 0;
+        p.t = t++;
+    }
+
+    __device__ bool next(Piece& p) {
+        if (stride) return next_rr(p);
+        if (i >= nseg || cur >= w_end) return false;
+        fill(p);
         p.new_x = first || j == 0;
         first = false;
         cur += gcw;
@@ -219,6 +302,36 @@ struct Walker {
         return true;
     }
 };
+
+// Exclusive block-wide scan of units_of(segs[b]) into segs[b].prefix; returns
+// the total.  Called by all THREADS threads; ends synchronised.
+template <typename UnitsFn>
+__device__ int32_t scan_segments(SegEntry* segs, int32_t nseg, int32_t* warp_sums, UnitsFn units_of) {
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    int32_t running = 0;
+    for (int32_t base = 0; base < nseg; base += THREADS) {
+        const int32_t b = base + tid;
+        const int32_t units = b < nseg ? units_of(segs[b]) : 0;
+        int32_t v = units;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += t;
+        }
+        if (lane == 31) warp_sums[warp] = v;
+        __syncthreads();
+        int32_t warp_off = 0, total = 0;
+        for (int w = 0; w < THREADS / 32; ++w) {
+            if (w < warp) warp_off += warp_sums[w];
+            total += warp_sums[w];
+        }
+        if (b < nseg) segs[b].prefix = running + warp_off + v - units;
+        running += total;
+        __syncthreads();
+    }
+    if (nseg <= 0) __syncthreads();
+    return running;
+}
 
 // Index k of the largest output box (8 << k rows, k <= max_level) that fits in
 // `rows` (a positive multiple of 8).
@@ -242,11 +355,12 @@ __device__ __forceinline__ int32_t ring_place(int32_t& head, int32_t rows8, int3
 
 // ---------------------------------------------------------------- the kernel
 
-template <int OUT_BYTES, bool ADD>
+template <int OUT_DT, bool ADD>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ YMaps ymaps, Problem p, Geometry geo,
                        const __grid_constant__ Slices sl) {
+    constexpr int OUT_BYTES = OUT_DT == SGMV_F32 ? 4 : 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -254,6 +368,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     __shared__ uint32_t s_tmem_base;
     __shared__ int32_t s_total_units;
     __shared__ int32_t s_warp_sums[THREADS / 32];
+    __shared__ int32_t s_partial_pieces;
+    __shared__ SliceTable s_sl;
 
     const int tid = threadIdx.x;
     const int warp = tid / 32;
@@ -276,6 +392,12 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
 
     if (tid == 0) {
         s_abort = 0;
+        s_partial_pieces = 0;
+        for (int i = 0; i <= MAX_SLICES; ++i) s_sl.tile0[i] = sl.tile0[i];
+        for (int i = 0; i < MAX_SLICES; ++i) {
+            s_sl.off[i] = (int32_t)sl.off[i];
+            s_sl.N[i] = (int32_t)sl.N[i];
+        }
         for (int i = 0; i < SW; ++i) {
             mbar_init(smem_u32(&w_full[i]), 1);
             mbar_init(smem_u32(&w_empty[i]), 1);
@@ -327,42 +449,38 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     // Everything below may read memory written by the preceding kernel.
     grid_dependency_wait();
 
-    // Segment table: guards of the API applied, units counted, exclusive scan.
+    // Segment table: guards of the API applied.
     const int32_t nseg = (int32_t)p.batches;
-    int32_t running = 0;
-    for (int32_t base = 0; base < nseg; base += THREADS) {
-        const int32_t b = base + tid;
-        int32_t units = 0;
-        SegEntry e{0, 0, 0, 0};
-        if (b < nseg) {
-            const Segment s = load_segment(p, b);
-            e.row0 = (int32_t)s.row0;
-            e.rows = (int32_t)s.rows;
-            e.adapter = (int32_t)s.adapter;
+    for (int32_t b = tid; b < nseg; b += THREADS) {
+        const Segment s = load_segment(p, b);
+        segs[b] = SegEntry{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0};
+    }
+    __syncthreads();
+    // Pieces per segment, and how many belong to partial (< 128-row) blocks.
+    int32_t my_partial = 0;
+    for (int32_t b = tid; b < nseg; b += THREADS)
+        if (segs[b].rows % BM) my_partial += geo.n_tiles;
+    if (my_partial) atomicAdd(&s_partial_pieces, my_partial);
+    const int32_t n_tiles = geo.n_tiles;
+    const int32_t total_pieces = scan_segments(segs, nseg, s_warp_sums, [&](const SegEntry& e) {
+        return (e.rows + BM - 1) / BM * n_tiles;
+    });
+    // Round-robin when long and short pieces are mixed: equal-weight ranges of
+    // the piece sequence then split unevenly, while every CTA's round-robin
+    // share is a fair sample.  With pieces all alike, contiguous ranges are
+    // already even and keep each CTA's x block in use across its n-tiles.
+    const int32_t partial = s_partial_pieces;   // complete: scan_segments synchronises
+    const bool rr = geo.rr && partial > 0 && 2 * partial <= total_pieces;
+    int32_t running = total_pieces;
+    if (!rr) {
+        const int32_t wmin = geo.wmin, wfix = geo.wfix;
+        running = scan_segments(segs, nseg, s_warp_sums, [&](const SegEntry& e) {
             const int32_t G = (e.rows + GROUP - 1) / GROUP;
-            if (G > 0) {
-                const int32_t full = (G - 1) / GROUPS_PER_BLOCK;          // full 128-row blocks
-                const int32_t last = G - full * GROUPS_PER_BLOCK;         // groups of the last block
-                units = (full * max(GROUPS_PER_BLOCK, geo.wmin) + max(last, geo.wmin)) * geo.n_tiles;
-            }
-        }
-        int32_t v = units;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += t;
-        }
-        if (lane == 31) s_warp_sums[warp] = v;
-        __syncthreads();
-        int32_t warp_off = 0, total = 0;
-        for (int w = 0; w < THREADS / 32; ++w) {
-            if (w < warp) warp_off += s_warp_sums[w];
-            total += s_warp_sums[w];
-        }
-        e.prefix = running + warp_off + v - units;
-        if (b < nseg) segs[b] = e;
-        running += total;
-        __syncthreads();
+            if (G == 0) return 0;
+            const int32_t full = (G - 1) / GROUPS_PER_BLOCK;          // full 128-row blocks
+            const int32_t last = G - full * GROUPS_PER_BLOCK;         // groups of the last block
+            return (full * max(GROUPS_PER_BLOCK, wmin) + max(last, wmin) + (full + 1) * wfix) * n_tiles;
+        });
     }
     if (tid == 0) s_total_units = running;
     grid_dependents_launch();
@@ -376,11 +494,15 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     const int32_t U = s_total_units;
     Walker walk;
     walk.segs = segs;
-    walk.tile0 = sl.tile0;
+    walk.st = &s_sl;
     walk.nseg = nseg;
     walk.n_tiles = geo.n_tiles;
     walk.wmin = geo.wmin;
-    walk.seek((int32_t)(((int64_t)U * blockIdx.x) / gridDim.x), (int32_t)(((int64_t)U * (blockIdx.x + 1)) / gridDim.x));
+    walk.wfix = geo.wfix;
+    if (rr)
+        walk.seek_rr((int32_t)blockIdx.x, (int32_t)gridDim.x);
+    else
+        walk.seek((int32_t)(((int64_t)U * blockIdx.x) / gridDim.x), (int32_t)(((int64_t)U * (blockIdx.x + 1)) / gridDim.x));
 
     volatile int* abort_flag = &s_abort;
     const bool w_bf16 = geo.w_is_bf16 != 0;
@@ -459,11 +581,10 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 ends[t % RING_PIECES] = head;
                 const uint32_t bar = smem_u32(&y_full[t % RING_PIECES]);
                 if (ADD) {
-                    const int ncols = min(BN, (int)(sl.N[pc.slice] - pc.n0));
-                    const int nch = (ncols + CC - 1) / CC;
+                    const int nch = (pc.ncols + CC - 1) / CC;
                     mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
                     const uint32_t ring = smem_u32(smem + geo.off_y);
-                    const int32_t xcol0 = (int32_t)(sl.off[pc.slice] + pc.n0);
+                    const int32_t xcol0 = pc.col0;
                     for (int c = 0; c < nch; ++c) {
                         for (int r = 0; r < rows8;) {
                             const int k = box_level(rows8 - r, NUM_YMAPS - 1);
@@ -567,7 +688,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         const int grp = (warp - EPI_WARP0) / 4;  // this warp's group takes pieces t % EPI_GROUPS == grp
         const int r = q * 32 + lane;             // block row of this thread
         const int ri = r % GROUP;
-        const bool out_bf16 = p.out_dt == SGMV_BF16;
+        constexpr bool out_bf16 = OUT_DT == SGMV_BF16;
         Piece pc;
         int32_t t = 0, head = 0;
         while (walk.next(pc)) {
@@ -585,8 +706,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                            DEVERR_TIMEOUT_EPILOGUE))
                 break;
             const int full_end = pc.rows & ~(GROUP - 1);
-            const int ncols = min(BN, (int)(sl.N[pc.slice] - pc.n0));
-            const int64_t col0 = sl.off[pc.slice] + pc.n0;   // first output column of the piece
+            const int ncols = pc.ncols;
+            const int64_t col0 = pc.col0;   // first output column of the piece
             const int pr = r - pc.shift;        // this thread's row within the piece
             const bool valid = pr >= 0 && pr < pc.rows;
             // rows past the last whole group go straight to global memory from registers
@@ -677,7 +798,9 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             __syncwarp();
             ++t;
         }
-        if (lane == 0) bulk_wait_all();
+        // the stores must have read shared memory before the CTA exits; the
+        // writes themselves complete with the grid
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
     }
 
@@ -723,9 +846,11 @@ struct Plan {
     Slices sl;
 };
 
-// Scheduling weight floor of a piece (8-row groups): a piece of a few rows
-// costs about as much pipeline time as one of several groups.
+// Scheduling weight of a piece = max(its 8-row groups of output, a floor) + a
+// fixed part: its B tile's bytes in units of one group's output bytes, plus
+// PIECE_FIXED_GROUPS for the per-piece pipeline work (MMA, barriers, TMA issue).
 constexpr int PIECE_WEIGHT_FLOOR = 16;
+constexpr int PIECE_FIXED_GROUPS = 0;
 
 // Shared-memory layout: an output ring of at least 4, else 3, 2, 1 whole
 // 128-row pieces, with the deepest B pipeline that leaves it room.
@@ -779,7 +904,7 @@ inline bool slice_ok(const Problem& p) {
     if (!aligned16(p.x) || !aligned16(p.w) || !aligned16(p.out)) return false;
     if ((p.H * so) % 16 || (p.off * so) % 16 || (p.N * so) % 16) return false;
     if (p.batches > SEG_CAP) return false;
-    if (p.out_rows >= (int64_t(1) << 31) || p.x_rows >= (int64_t(1) << 31) || p.off + p.N >= (int64_t(1) << 32))
+    if (p.out_rows >= (int64_t(1) << 31) || p.x_rows >= (int64_t(1) << 31) || p.off + p.N >= (int64_t(1) << 31))
         return false;
     if (p.lora_num >= (int64_t(1) << 31)) return false;
     return true;
@@ -812,7 +937,9 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     const int64_t n_tiles = sl.tile0[nsl];
     const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int64_t max_pieces = (t_lim / BM + p.batches + 1) * n_tiles;
-    const int64_t weight_bound = (t_lim / GROUP + p.batches + 1) * n_tiles + PIECE_WEIGHT_FLOOR * max_pieces;
+    const int64_t group_bytes = (int64_t)GROUP * BN * so * (p.add ? 2 : 1);
+    const int64_t wfix = (BN * p.K * 2 + group_bytes - 1) / group_bytes + PIECE_FIXED_GROUPS;
+    const int64_t weight_bound = (t_lim / GROUP + p.batches + 1) * n_tiles + (wfix + PIECE_WEIGHT_FLOOR) * max_pieces;
     if (weight_bound >= (int64_t(1) << 31)) return false;
 
     Geometry& g = out->geo;
@@ -823,6 +950,10 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     g.n_tiles = (int32_t)n_tiles;
     g.w_is_bf16 = p.w_dt == SGMV_BF16;
     g.wmin = PIECE_WEIGHT_FLOOR;
+    // Round-robin pieces are allowed unless x must be rounded to the weights'
+    // dtype: that is done once per x block, so a CTA keeps a block's n-tiles.
+    g.rr = g.convert_x ? 0 : 1;
+    g.wfix = (int32_t)wfix;
     // B tile: K in blocks of 64 columns, then at most one each of 32, 16, 8
     {
         int k0 = 0, off = 0, nb = 0;
@@ -931,9 +1062,9 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     return true;
 }
 
-template <int OUT_BYTES, bool ADD>
+template <int OUT_DT, bool ADD>
 int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
-    auto kern = tc_expand_slice_kernel<OUT_BYTES, ADD>;
+    auto kern = tc_expand_slice_kernel<OUT_DT, ADD>;
     static std::atomic<bool> configured{false};
     if (!configured.load()) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -966,10 +1097,17 @@ int launch_tc(const Problem* ps, int nsl, int sm_count, cudaStream_t stream) {
     tc::Plan pl;
     if (!tc::make_plan(ps, nsl, sm_count, &pl)) return SGMV_ERR_VARIANT;
     const Problem& p = ps[0];
-    if (tc::elem_bytes(p.out_dt) == 4) {
-        return p.add ? tc::launch_instance<4, true>(pl, p, stream) : tc::launch_instance<4, false>(pl, p, stream);
+    switch (p.out_dt) {
+        case SGMV_F32:
+            return p.add ? tc::launch_instance<SGMV_F32, true>(pl, p, stream)
+                         : tc::launch_instance<SGMV_F32, false>(pl, p, stream);
+        case SGMV_BF16:
+            return p.add ? tc::launch_instance<SGMV_BF16, true>(pl, p, stream)
+                         : tc::launch_instance<SGMV_BF16, false>(pl, p, stream);
+        default:
+            return p.add ? tc::launch_instance<SGMV_F16, true>(pl, p, stream)
+                         : tc::launch_instance<SGMV_F16, false>(pl, p, stream);
     }
-    return p.add ? tc::launch_instance<2, true>(pl, p, stream) : tc::launch_instance<2, false>(pl, p, stream);
 }
 
 }  // namespace sgmv

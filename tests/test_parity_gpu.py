@@ -112,6 +112,36 @@ def test_ranks(K, variant):
     check_full(p, variant)
 
 
+# The tensor-core kernel hands pieces out round-robin when full 128-row blocks
+# and partial ones are mixed (at most half of the pieces partial), and in
+# contiguous ranges otherwise; these cases put each mode through ranks, dtypes
+# and a segment table longer than one pass of its block-wide scan.
+MIXED_BLOCKS = [256, 3, 384, 130, 1, 128]          # 7 full blocks, 3 partial: round-robin
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("K,out_dt", [(8, "bf16"), (16, "f16"), (24, "bf16"), (64, "f32"), (128, "bf16")])
+def test_mixed_block_lengths(K, out_dt, variant):
+    p = gen.custom(seed=40 + K, lengths=MIXED_BLOCKS, K=K, N=200, H=456, offset=128, num_adapters=4,
+                   x_dt="f16" if out_dt == "f16" else "bf16", w_dt="f16" if out_dt == "f16" else "bf16",
+                   out_dt=out_dt)
+    check_full(p, variant)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("share_short", [0.1, 0.9])
+def test_many_segments(share_short, variant):
+    """800 segments (more than one 352-wide scan pass): 10% short segments picks
+    round-robin, 90% short picks contiguous ranges."""
+    rng = np.random.default_rng(int(share_short * 100))
+    short = rng.random(800) < share_short
+    lengths = np.where(short, rng.integers(1, 20, 800), 128 * rng.integers(1, 3, 800))
+    idx = rng.integers(-1, 6, 800)
+    p = gen.custom(seed=11, lengths=lengths.tolist(), K=16, N=64, H=192, offset=64, num_adapters=6,
+                   idx=idx.tolist())
+    check_full(p, variant)
+
+
 @pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("x_dt", gen.ALL_DTYPES)
 @pytest.mark.parametrize("w_dt", gen.HALF_DTYPES)

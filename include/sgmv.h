@@ -90,6 +90,7 @@ enum {
     SGMV_ERR_VARIANT = -13,          /* the forced kernel variant cannot run this call */
     SGMV_ERR_NUM_SLICES = -14,       /* num_slices outside [1, SGMV_MAX_SLICES] */
     SGMV_ERR_SLICE_OVERLAP = -15,    /* two non-empty slices of one call share a column */
+    SGMV_ERR_OUT_WIDTH = -16,        /* sgmv_expand: out.shape[1] != lora_b.shape[-2] */
     SGMV_ERR_CUDA = -20,             /* a CUDA runtime call failed */
     SGMV_ERR_LAUNCH = -21            /* a kernel launch failed */
 };
@@ -98,7 +99,8 @@ enum {
 enum {
     SGMV_VARIANT_AUTO = 0,
     SGMV_VARIANT_SIMT = 1,   /* generic CUDA-core kernel: any strides, rank, alignment */
-    SGMV_VARIANT_TC = 2      /* tcgen05 tensor-core kernel with TMA staging */
+    SGMV_VARIANT_TC = 2,     /* tcgen05 tensor-core kernel with TMA staging */
+    SGMV_VARIANT_DECODE = 3  /* bgmv_expand_slice's one-token-per-row kernel (vector loads) */
 };
 
 /*
@@ -177,6 +179,44 @@ SGMV_API int sgmv_plan_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor*
                           const sgmv_tensor* out, const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
                           const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len,
                           const int64_t* slice_offsets, int add_inputs, int* variant, int* launches);
+
+/*
+ * sgmv_expand -- the standard SGMV expand that the expand-slice operation
+ * extends ("Implementation: Predibase Lorax SGMV Expand Slice Kernel",
+ * Description): the whole output row is the slice, i.e. the operation above
+ * with slice_offset = 0 and slice_size = N, where N = lora_b.shape[-2] must
+ * equal out.shape[1] (else SGMV_ERR_OUT_WIDTH).  Every other argument, rule and
+ * status is as for sgmv_expand_slice.
+ */
+SGMV_API int sgmv_expand(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+                const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+                int64_t batches, int64_t max_seq_len, int add_inputs, void* stream);
+
+/*
+ * bgmv_expand_slice -- the fixed-length counterpart of the expand-slice
+ * operation (the page calls SGMV expand-slice "the variable-length sequence
+ * counterpart to the BGMV expand slice kernel", Description): every row b <
+ * batches is one token with its own adapter a = lora_idx[b],
+ *
+ *     out[b, off + n] = (add_inputs ? out[b, off + n] : 0) + sum_k x^[b, k] * B[a][n, k]
+ *
+ * which is sgmv_expand_slice with seq_start[b] = b and seq_len[b] = 1.  Same
+ * tensors, dtypes, rounding, guards and statuses as sgmv_expand_slice, without
+ * seq_start, seq_len and max_seq_len; rows at or beyond the row count of
+ * inputs or of out are skipped.  Runs a kernel made for one token per row
+ * (SGMV_VARIANT_DECODE) when B and x have unit column stride, K is a multiple
+ * of 8 no larger than 256 and their rows start on 16-byte boundaries;
+ * otherwise the generic CUDA-core kernel.
+ */
+SGMV_API int bgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+                      const sgmv_tensor* lora_idx, int64_t batches, int64_t slice_offset, int64_t slice_size,
+                      int add_inputs, void* stream);
+
+/* bgmv_plan -- validate as bgmv_expand_slice does; *variant receives the
+ * kernel variant a call would launch (0 when nothing launches). */
+SGMV_API int bgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+              const sgmv_tensor* lora_idx, int64_t batches, int64_t slice_offset, int64_t slice_size,
+              int add_inputs, int* variant);
 
 /*
  * sgmv_validate_metadata -- check the VALUES of the metadata on the device and

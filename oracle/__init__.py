@@ -132,6 +132,31 @@ def expand_slice(x, x_dt, w, w_dt, out, out_dt, seq_start, seq_len, lora_idx,
     return y
 
 
+def expand(x, x_dt, w, w_dt, out, out_dt, seq_start, seq_len, lora_idx, add_inputs, batches=None,
+           nthreads=1, return_pre=False):
+    """The standard SGMV expand that the slice operation extends ("Implementation:
+    Predibase Lorax SGMV Expand Slice Kernel", Description): the whole output
+    row is the slice, so this is expand_slice with slice_offset 0 and
+    slice_size = lora_b's N, which must equal out's width."""
+    N = w.shape[-2]
+    assert out.shape[1] == N, "plain expand writes whole rows: out's width must equal lora_b's N"
+    return expand_slice(x, x_dt, w, w_dt, out, out_dt, seq_start, seq_len, lora_idx, 0, N, add_inputs,
+                        batches=batches, nthreads=nthreads, return_pre=return_pre)
+
+
+def bgmv_expand_slice(x, x_dt, w, w_dt, out, out_dt, lora_idx, slice_offset, slice_size, add_inputs,
+                      batches=None, nthreads=1, return_pre=False):
+    """BGMV expand-slice, the fixed-length counterpart the same page names
+    (Description): row b (b < batches) is one token with adapter lora_idx[b],
+    i.e. expand_slice with seq_start[b] = b and seq_len[b] = 1."""
+    li = np.asarray(lora_idx, dtype=np.int64)
+    B = len(li) if batches is None else int(batches)
+    starts = np.arange(B, dtype=np.int64)
+    lens = np.ones(B, dtype=np.int64)
+    return expand_slice(x, x_dt, w, w_dt, out, out_dt, starts, lens, li[:B], slice_offset, slice_size,
+                        add_inputs, batches=B, nthreads=nthreads, return_pre=return_pre)
+
+
 def run_problem(p, nthreads=1, return_pre=False, out=None, call=0):
     """Run the oracle on a `sgmv_inputs.Problem` (one of its slice calls)."""
     c = p.calls[call]

@@ -18,6 +18,9 @@ for every sequence b with ``lora_indices_tensor[b] != -1`` and token m, with
 ``sgmv_expand_multi_slice`` updates several disjoint slices of one fused
 output (the QKV or gate/up projections the page's Usage section names) in a
 single call, which the page's Description anticipates as a fused operator.
+``sgmv_expand`` is the standard expand the slice operation extends (the whole
+output row is the slice), and ``bgmv_expand_slice`` its fixed-length
+counterpart with one token per row (both named in the page's Description).
 """
 import ctypes
 
@@ -25,10 +28,12 @@ import torch
 
 from . import _abi
 
-__all__ = ["sgmv_expand_slice", "sgmv_expand_multi_slice", "plan", "plan_multi_slice", "validate_metadata", "set_variant", "device_error",
-           "SgmvError", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "library_path"]
+__all__ = ["sgmv_expand_slice", "sgmv_expand_multi_slice", "sgmv_expand", "bgmv_expand_slice", "plan",
+           "plan_multi_slice", "bgmv_plan", "validate_metadata", "set_variant", "device_error", "SgmvError",
+           "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "VARIANT_DECODE", "library_path"]
 
 VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC = _abi.VARIANT_AUTO, _abi.VARIANT_SIMT, _abi.VARIANT_TC
+VARIANT_DECODE = _abi.VARIANT_DECODE
 library_path = _abi.LIB_PATH
 
 _DTYPES = {torch.float16: _abi.F16, torch.bfloat16: _abi.BF16, torch.float32: _abi.F32,
@@ -78,6 +83,56 @@ def sgmv_expand_slice(inputs, lora_b_weights, output_tensor, b_seq_start_loc, se
     if rc != 0:
         raise SgmvError(rc, "sgmv_expand_slice")
     return output_tensor
+
+
+def sgmv_expand(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor,
+                lora_indices_tensor, batches, max_seq_length, add_inputs=False):
+    """In-place standard SGMV expand: ``output_tensor`` is as wide as the slice
+    (``lora_b_weights.shape[-2]``), which starts at column 0."""
+    d = _args(inputs, lora_b_weights, output_tensor, b_seq_start_loc, seq_len_tensor,
+              lora_indices_tensor)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_expand(*[ctypes.byref(x) for x in d], int(batches), int(max_seq_length),
+                              int(bool(add_inputs)), _stream_handle(output_tensor.device))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_expand")
+    return output_tensor
+
+
+def _bgmv_args(inputs, lora_b_weights, output_tensor, lora_indices_tensor):
+    ts = [inputs, lora_b_weights, output_tensor, lora_indices_tensor]
+    for t in ts:
+        if not t.is_cuda or t.device != output_tensor.device:
+            raise ValueError("all tensors must be CUDA tensors on the same device")
+    return [_desc(t) for t in ts]
+
+
+def bgmv_expand_slice(inputs, lora_b_weights, output_tensor, lora_indices_tensor, slice_offset, slice_size,
+                      add_inputs=False, batches=None):
+    """In-place BGMV expand-slice: row b of ``inputs`` is one token with adapter
+    ``lora_indices_tensor[b]``; ``batches`` defaults to ``inputs.shape[0]``."""
+    batches = inputs.shape[0] if batches is None else batches
+    d = _bgmv_args(inputs, lora_b_weights, output_tensor, lora_indices_tensor)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.bgmv_expand_slice(*[ctypes.byref(x) for x in d], int(batches), int(slice_offset),
+                                    int(slice_size), int(bool(add_inputs)), _stream_handle(output_tensor.device))
+    if rc != 0:
+        raise SgmvError(rc, "bgmv_expand_slice")
+    return output_tensor
+
+
+def bgmv_plan(inputs, lora_b_weights, output_tensor, lora_indices_tensor, slice_offset, slice_size,
+              add_inputs=False, batches=None) -> int:
+    """Kernel variant a bgmv_expand_slice call with these arguments would launch (0 = none)."""
+    batches = inputs.shape[0] if batches is None else batches
+    d = _bgmv_args(inputs, lora_b_weights, output_tensor, lora_indices_tensor)
+    v = ctypes.c_int(0)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.bgmv_plan(*[ctypes.byref(x) for x in d], int(batches), int(slice_offset), int(slice_size),
+                            int(bool(add_inputs)), ctypes.byref(v))
+    if rc != 0:
+        raise SgmvError(rc, "bgmv_plan")
+    return v.value
 
 
 def _multi_args(inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor,

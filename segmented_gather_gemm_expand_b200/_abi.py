@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(HERE, "libsgmv.so")
 F16, BF16, F32, I32, I64 = 0, 1, 2, 3, 4
 
 SGMV_OK = 0
-VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC = 0, 1, 2
+VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC, VARIANT_DECODE = 0, 1, 2, 3
 
 STATUS_NAMES = {
     0: "SGMV_OK", -1: "SGMV_ERR_NULL_ARG", -2: "SGMV_ERR_DTYPE", -3: "SGMV_ERR_NDIM",
@@ -21,6 +21,7 @@ STATUS_NAMES = {
     -7: "SGMV_ERR_OUT_NOT_CONTIGUOUS", -8: "SGMV_ERR_SLICE_RANGE", -9: "SGMV_ERR_BATCHES",
     -10: "SGMV_ERR_SHAPE", -11: "SGMV_ERR_STRIDE", -12: "SGMV_ERR_TOO_LARGE",
     -13: "SGMV_ERR_VARIANT", -14: "SGMV_ERR_NUM_SLICES", -15: "SGMV_ERR_SLICE_OVERLAP",
+    -16: "SGMV_ERR_OUT_WIDTH",
     -20: "SGMV_ERR_CUDA", -21: "SGMV_ERR_LAUNCH",
 }
 MAX_SLICES = 4
@@ -68,6 +69,12 @@ def load():
     lib.sgmv_plan_multi_slice.restype = i32
     lib.sgmv_plan_multi_slice.argtypes = [P, PP, i32, P, P, P, P, i64, i64, I64P, i32,
                                           ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.sgmv_expand.restype = i32
+    lib.sgmv_expand.argtypes = [P, P, P, P, P, P, i64, i64, i32, vp]
+    lib.bgmv_expand_slice.restype = i32
+    lib.bgmv_expand_slice.argtypes = [P, P, P, P, i64, i64, i64, i32, vp]
+    lib.bgmv_plan.restype = i32
+    lib.bgmv_plan.argtypes = [P, P, P, P, i64, i64, i64, i32, ctypes.POINTER(i32)]
     lib.sgmv_validate_metadata.restype = i32
     lib.sgmv_validate_metadata.argtypes = [P, P, P, i64, i64, i64, vp, vp]
     lib.sgmv_status_string.restype = ctypes.c_char_p

@@ -11,10 +11,14 @@
 
 namespace sgmv {
 
-// One metadata vector (seq_start, seq_len or lora_idx): i32 or i64, any stride.
+// One metadata vector (seq_start, seq_len or lora_idx): i32 or i64, any stride,
+// or an implicit vector with no memory behind it: element b is b (META_IOTA)
+// or 1 (META_ONE), which describes one-token rows (bgmv_expand_slice).
+constexpr int32_t META_IOTA = 100;
+constexpr int32_t META_ONE = 101;
 struct MetaVec {
     const void* ptr;
-    int32_t dtype;     // SGMV_I32 | SGMV_I64
+    int32_t dtype;     // SGMV_I32 | SGMV_I64 | META_IOTA | META_ONE
     int64_t stride;    // elements
 };
 
@@ -36,6 +40,8 @@ struct Problem {
 };
 
 __device__ __forceinline__ int64_t load_meta(const MetaVec& m, int64_t i) {
+    if (m.dtype == META_IOTA) return i;
+    if (m.dtype == META_ONE) return 1;
     if (m.dtype == SGMV_I64) return __ldg(reinterpret_cast<const long long*>(m.ptr) + i * m.stride);
     return (int64_t)__ldg(reinterpret_cast<const int*>(m.ptr) + i * m.stride);
 }

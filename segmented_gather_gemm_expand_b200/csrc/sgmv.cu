@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "bgmv.cuh"
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc.cuh"
@@ -189,6 +190,7 @@ int launch_simt(const Call& c, const DeviceInfo& dev, cudaStream_t stream) {
 int choose_variant(const Call& c, const DeviceInfo& dev, int forced) {
     const bool tc_ok = dev.cc_major == 10 && tc_supports(&c.p, 1);
     if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
+    if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;   // bgmv_expand_slice's kernel only
     if (forced == SGMV_VARIANT_TC) return tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
     return tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
 }
@@ -224,6 +226,7 @@ int validate_multi(const sgmv_tensor* x, const sgmv_tensor* const* ws, int num_s
 // slice, each with its own variant.  Returns the fused variant or a status.
 int choose_multi(const Call* calls, int n, const DeviceInfo& dev, int forced, bool* fused) {
     *fused = false;
+    if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;   // bgmv_expand_slice's kernel only
     if (forced != SGMV_VARIANT_SIMT && dev.cc_major == 10) {
         Problem ps[SGMV_MAX_SLICES];
         for (int i = 0; i < n; ++i) ps[i] = calls[i].p;
@@ -239,9 +242,100 @@ int choose_multi(const Call* calls, int n, const DeviceInfo& dev, int forced, bo
     return forced == SGMV_VARIANT_SIMT ? (int)SGMV_VARIANT_SIMT : 0;
 }
 
+// bgmv_expand_slice: the expand-slice validation with row b as a one-token
+// segment (start b, length 1); lora_idx stands in for the other two metadata
+// tensors in the shape checks, then they become implicit vectors.
+int validate_bgmv(const sgmv_tensor* x, const sgmv_tensor* w, const sgmv_tensor* out, const sgmv_tensor* idx,
+                  int64_t batches, int64_t slice_offset, int64_t slice_size, int add_inputs, Call* call) {
+    const int rc = validate_call(x, w, out, idx, idx, idx, batches, 1, slice_offset, slice_size, add_inputs, call);
+    if (rc) return rc;
+    call->p.start = MetaVec{nullptr, META_IOTA, 0};
+    call->p.len = MetaVec{nullptr, META_ONE, 0};
+    call->max_seq_len = 1;
+    return SGMV_OK;
+}
+
+bool bgmv_fast_ok(const Problem& p) {
+    if (p.K < 8 || p.K > BGMV_MAX_K || p.K % 8 != 0 || p.w_ks != 1) return false;
+    if ((reinterpret_cast<uintptr_t>(p.w) & 15) || (p.w_ns * 2) % 16) return false;
+    if (p.lora_num > 1 && (p.w_as * 2) % 16) return false;
+    if ((p.N + BGMV_COLS - 1) / BGMV_COLS > 0x7fffffff) return false;
+    return true;
+}
+
+int choose_bgmv(const Call& c, int forced) {
+    const bool fast = bgmv_fast_ok(c.p);
+    if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
+    if (forced == SGMV_VARIANT_TC) return SGMV_ERR_VARIANT;
+    if (forced == SGMV_VARIANT_DECODE) return fast ? (int)SGMV_VARIANT_DECODE : (int)SGMV_ERR_VARIANT;
+    return fast ? SGMV_VARIANT_DECODE : SGMV_VARIANT_SIMT;
+}
+
+template <int OUT_DT>
+int launch_bgmv_dt(const Problem& p, dim3 grid, cudaStream_t stream) {
+    if (p.add) bgmv_expand_kernel<OUT_DT, true><<<grid, BGMV_THREADS, 0, stream>>>(p);
+    else bgmv_expand_kernel<OUT_DT, false><<<grid, BGMV_THREADS, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SGMV_OK : SGMV_ERR_LAUNCH;
+}
+
+int launch_bgmv(const Call& c, cudaStream_t stream) {
+    const Problem& p = c.p;
+    dim3 grid((unsigned)((p.N + BGMV_COLS - 1) / BGMV_COLS), (unsigned)(p.batches < 65535 ? p.batches : 65535));
+    switch (p.out_dt) {
+        case SGMV_F32: return launch_bgmv_dt<SGMV_F32>(p, grid, stream);
+        case SGMV_BF16: return launch_bgmv_dt<SGMV_BF16>(p, grid, stream);
+        default: return launch_bgmv_dt<SGMV_F16>(p, grid, stream);
+    }
+}
+
 }  // namespace
 
 extern "C" {
+
+int sgmv_expand(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+                const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+                int64_t batches, int64_t max_seq_len, int add_inputs, void* stream) {
+    int rc;
+    if ((rc = check_basic(lora_b))) return rc;
+    if ((rc = check_basic(out))) return rc;
+    if (lora_b->ndim != 3 && lora_b->ndim != 4) return SGMV_ERR_NDIM;
+    if (out->ndim != 2) return SGMV_ERR_NDIM;
+    const int64_t N = lora_b->shape[lora_b->ndim - 2];
+    if (out->shape[1] != N) return SGMV_ERR_OUT_WIDTH;
+    return sgmv_expand_slice(inputs, lora_b, out, seq_start, seq_len, lora_idx, batches, max_seq_len, 0, N,
+                             add_inputs, stream);
+}
+
+int bgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+                      const sgmv_tensor* lora_idx, int64_t batches, int64_t slice_offset, int64_t slice_size,
+                      int add_inputs, void* stream) {
+    Call c;
+    int rc = validate_bgmv(inputs, lora_b, out, lora_idx, batches, slice_offset, slice_size, add_inputs, &c);
+    if (rc) return rc;
+    if (c.empty) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    const int v = choose_bgmv(c, g_forced_variant.load());
+    if (v < 0) return v;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (v == SGMV_VARIANT_DECODE) return launch_bgmv(c, st);
+    return launch_simt(c, dev, st);
+}
+
+int bgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
+              const sgmv_tensor* lora_idx, int64_t batches, int64_t slice_offset, int64_t slice_size,
+              int add_inputs, int* variant) {
+    if (!variant) return SGMV_ERR_NULL_ARG;
+    *variant = 0;
+    Call c;
+    const int rc = validate_bgmv(inputs, lora_b, out, lora_idx, batches, slice_offset, slice_size, add_inputs, &c);
+    if (rc) return rc;
+    if (c.empty) return SGMV_OK;
+    const int v = choose_bgmv(c, g_forced_variant.load());
+    if (v < 0) return v;
+    *variant = v;
+    return SGMV_OK;
+}
 
 int sgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
                       const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
@@ -252,9 +346,11 @@ int sgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, cons
                            slice_offset, slice_size, add_inputs, &c);
     if (rc) return rc;
     if (c.empty) return SGMV_OK;
+    const int forced = g_forced_variant.load();
+    if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;   // bgmv_expand_slice's kernel only
     DeviceInfo dev;
     if ((rc = device_info(&dev))) return rc;
-    const int v = choose_variant(c, dev, g_forced_variant.load());
+    const int v = choose_variant(c, dev, forced);
     if (v < 0) return v;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (v == SGMV_VARIANT_TC) return launch_tc(&c.p, 1, dev.sm_count, st);
@@ -272,9 +368,11 @@ int sgmv_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_t
                            slice_offset, slice_size, add_inputs, &c);
     if (rc) return rc;
     if (c.empty) return SGMV_OK;
+    const int forced = g_forced_variant.load();
+    if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;   // bgmv_expand_slice's kernel only
     DeviceInfo dev;
     if ((rc = device_info(&dev))) return rc;
-    const int v = choose_variant(c, dev, g_forced_variant.load());
+    const int v = choose_variant(c, dev, forced);
     if (v < 0) return v;
     *variant = v;
     return SGMV_OK;
@@ -290,6 +388,7 @@ int sgmv_expand_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const*
                             slice_offsets, add_inputs, calls, &n);
     if (rc) return rc;
     if (n == 0) return SGMV_OK;
+    if (g_forced_variant.load() == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;
     DeviceInfo dev;
     if ((rc = device_info(&dev))) return rc;
     const int forced = g_forced_variant.load();
@@ -323,6 +422,7 @@ int sgmv_plan_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const* l
                             slice_offsets, add_inputs, calls, &n);
     if (rc) return rc;
     if (n == 0) return SGMV_OK;
+    if (g_forced_variant.load() == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;
     DeviceInfo dev;
     if ((rc = device_info(&dev))) return rc;
     bool fused = false;
@@ -378,6 +478,7 @@ const char* sgmv_status_string(int code) {
         case SGMV_ERR_VARIANT: return "the forced kernel variant cannot run this call";
         case SGMV_ERR_NUM_SLICES: return "num_slices outside [1, SGMV_MAX_SLICES]";
         case SGMV_ERR_SLICE_OVERLAP: return "two slices of a multi-slice call overlap";
+        case SGMV_ERR_OUT_WIDTH: return "sgmv_expand: out.shape[1] != lora_b.shape[-2]";
         case SGMV_ERR_CUDA: return "a CUDA runtime call failed";
         case SGMV_ERR_LAUNCH: return "kernel launch failed";
         default: return "unknown status";
@@ -385,7 +486,8 @@ const char* sgmv_status_string(int code) {
 }
 
 int sgmv_set_variant(int variant) {
-    if (variant != SGMV_VARIANT_AUTO && variant != SGMV_VARIANT_SIMT && variant != SGMV_VARIANT_TC)
+    if (variant != SGMV_VARIANT_AUTO && variant != SGMV_VARIANT_SIMT && variant != SGMV_VARIANT_TC &&
+        variant != SGMV_VARIANT_DECODE)
         return SGMV_ERR_VARIANT;
     return g_forced_variant.exchange(variant);
 }

@@ -21,7 +21,7 @@ def declared_functions():
     for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
         if fn.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fn)).read()
-            names += re.findall(r"SGMV_API\s+[\w\s\*]+?\b(sgmv_\w+)\s*\(", text)
+            names += re.findall(r"SGMV_API\s+[\w\s\*]+?\b((?:sgmv|bgmv)_\w+)\s*\(", text)
     return names
 
 
@@ -219,3 +219,56 @@ def test_multi_slice_empty_needs_no_device():
     assert call_multi(good_args(batches=0), [wslice(128), wslice(128)], [0, 128]) == 0
     # an empty slice inside a non-empty one overlaps nothing
     assert call_multi(good_args(batches=0), [wslice(128), wslice(0)], [0, 64]) == 0
+
+
+# ------------------------------------------------------------ plain expand and BGMV
+
+def test_plain_expand_rejects_a_partial_width_output():
+    lib = _abi.load()
+    a = good_args()          # out is wider than lora_b's N: a slice call, not a plain expand
+    r = ctypes.byref
+    rc = lib.sgmv_expand(r(a["x"]), r(a["w"]), r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]),
+                         a["batches"], a["max_seq_len"], a["add"], None)
+    assert rc == _abi.STATUS["SGMV_ERR_OUT_WIDTH"]
+    w2 = _abi.make_tensor(FAKE, _abi.BF16, (A, N), (N, 1))
+    assert lib.sgmv_expand(r(a["x"]), r(w2), r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]), 4, 7, 0, None) == \
+        _abi.STATUS["SGMV_ERR_NDIM"]
+    assert lib.sgmv_expand(r(a["x"]), None, r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]), 4, 7, 0, None) == \
+        _abi.STATUS["SGMV_ERR_NULL_ARG"]
+
+
+BGMV_BAD = {
+    "idx_shorter_than_batches": (dict(batches=5), "SGMV_ERR_BATCHES"),
+    "slice_past_width": (dict(off=300), "SGMV_ERR_SLICE_RANGE"),
+    "slice_size_mismatch": (dict(size=64), "SGMV_ERR_SLICE_SIZE"),
+    "w_dtype_f32": (dict(w=_abi.make_tensor(FAKE, _abi.F32, (A, N, K), (N * K, K, 1))), "SGMV_ERR_DTYPE"),
+    "idx_dtype_f16": (dict(i=_abi.make_tensor(FAKE, _abi.F16, (B,), (1,))), "SGMV_ERR_DTYPE"),
+    "rank_mismatch": (dict(x=_abi.make_tensor(FAKE, _abi.BF16, (T, 8), (8, 1))), "SGMV_ERR_RANK_MISMATCH"),
+    "negative_batches": (dict(batches=-2), "SGMV_ERR_BATCHES"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(BGMV_BAD))
+def test_bgmv_invalid_arguments_fail_before_launch(case):
+    lib = _abi.load()
+    over, code = BGMV_BAD[case]
+    a = good_args(**over)
+    r = ctypes.byref
+    rc = lib.bgmv_expand_slice(r(a["x"]), r(a["w"]), r(a["out"]), r(a["i"]), a["batches"], a["off"], a["size"],
+                               a["add"], None)
+    assert rc == _abi.STATUS[code]
+    v = ctypes.c_int(-1)
+    rc = lib.bgmv_plan(r(a["x"]), r(a["w"]), r(a["out"]), r(a["i"]), a["batches"], a["off"], a["size"],
+                       a["add"], r(v))
+    assert rc == _abi.STATUS[code] and v.value == 0
+
+
+def test_decode_variant_is_only_for_bgmv():
+    """Forcing the one-token kernel makes expand-slice calls report SGMV_ERR_VARIANT (before any launch)."""
+    lib = _abi.load()
+    prev = lib.sgmv_set_variant(3)
+    try:
+        a = good_args()
+        assert call(a) == _abi.STATUS["SGMV_ERR_VARIANT"]
+    finally:
+        lib.sgmv_set_variant(prev)

@@ -51,6 +51,8 @@ WORKLOAD_TEXT = {
     "decode_mix": "decode-like mix: 256 seqs Zipf(1.2) in [1,64], rank 32, 256 distinct adapters "
                   "(10% -1), bf16, slice 5120 at 5120 of T x 15360, add_inputs",
     "tiny": "tiny: 4 seqs [4,6,3,7], rank 16, fp16, slice 128 at 128, overwrite",
+    "decode_bgmv": "decode step (bgmv_expand_slice): 256 one-token rows, 256 distinct adapters (10% -1), "
+                   "rank 32, bf16, slice 5120 at 5120 of 256 x 15360, add_inputs",
 }
 
 DT_SIZE = {"f16": 2, "bf16": 2, "f32": 4}
@@ -65,7 +67,7 @@ def call_accounting(p: gen.Problem, call: int):
     ok = (p.lora_idx >= 0) & (p.lora_idx < A) & (p.seq_len > 0) & (p.seq_start >= 0)
     rows = int(p.seq_len[ok].sum())
     adapters = len(np.unique(p.lora_idx[ok]))
-    meta = 3 * p.batches * (8 if p.meta_dt == "int64" else 4)
+    meta = (1 if p.op == "bgmv" else 3) * p.batches * (8 if p.meta_dt == "int64" else 4)
     sx, sw, so = DT_SIZE[p.x_dt], DT_SIZE[p.w_dt], DT_SIZE[p.out_dt]
     byts = rows * (K * sx + N * so * (2 if p.add_inputs else 1)) + adapters * N * K * sw + meta
     flops = 2 * N * K * rows
@@ -197,10 +199,15 @@ def make_calls(p, dev_tensors, sg_abi, stream_handle_fn):
 
     def run(c, stream):
         d, off, size = descs[c]
-        rc = lib.sgmv_expand_slice(*[ctypes.byref(t) for t in d], p.batches, p.max_seq_len, off, size,
-                                   int(p.add_inputs), ctypes.c_void_p(stream))
+        if p.op == "bgmv":   # x, B, out and lora_idx only: row b is one token
+            rc = lib.bgmv_expand_slice(ctypes.byref(d[0]), ctypes.byref(d[1]), ctypes.byref(d[2]),
+                                       ctypes.byref(d[5]), p.batches, off, size, int(p.add_inputs),
+                                       ctypes.c_void_p(stream))
+        else:
+            rc = lib.sgmv_expand_slice(*[ctypes.byref(t) for t in d], p.batches, p.max_seq_len, off, size,
+                                       int(p.add_inputs), ctypes.c_void_p(stream))
         if rc != 0:
-            raise sg.SgmvError(rc, "sgmv_expand_slice")
+            raise sg.SgmvError(rc, "bgmv_expand_slice" if p.op == "bgmv" else "sgmv_expand_slice")
     return run, descs
 
 
@@ -285,9 +292,13 @@ def bench_ours(args, rank, world, device):
     meta = [m.to(device) for m in hmeta]
     run, _ = make_calls(p, (x, ws, y, meta), _abi, None)
     ncalls = len(p.calls)
-    v_used = sg.plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, p.calls[0].slice_offset,
-                     p.calls[0].slice_size, p.add_inputs)
-    variant_name = {1: "simt", 2: "tc"}.get(v_used, str(v_used))
+    if p.op == "bgmv":
+        v_used = sg.bgmv_plan(x, ws[0], y, meta[2], p.calls[0].slice_offset, p.calls[0].slice_size,
+                              p.add_inputs)
+    else:
+        v_used = sg.plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, p.calls[0].slice_offset,
+                         p.calls[0].slice_size, p.add_inputs)
+    variant_name = {1: "simt", 2: "tc", 3: "decode"}.get(v_used, str(v_used))
 
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()

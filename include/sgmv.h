@@ -41,6 +41,7 @@
 #ifndef SGMV_H
 #define SGMV_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -90,7 +91,8 @@ enum {
     SGMV_ERR_VARIANT = -13,          /* the forced kernel variant cannot run this call */
     SGMV_ERR_NUM_SLICES = -14,       /* num_slices outside [1, SGMV_MAX_SLICES] */
     SGMV_ERR_SLICE_OVERLAP = -15,    /* two non-empty slices of one call share a column */
-    SGMV_ERR_OUT_WIDTH = -16,        /* sgmv_expand: out.shape[1] != lora_b.shape[-2] */
+    SGMV_ERR_OUT_WIDTH = -16,        /* sgmv_expand / sgmv_shrink: out.shape[1] != lora_b/lora_a.shape[-2] */
+    SGMV_ERR_WORKSPACE = -17,        /* sgmv_shrink: workspace not 16-byte aligned */
     SGMV_ERR_CUDA = -20,             /* a CUDA runtime call failed */
     SGMV_ERR_LAUNCH = -21            /* a kernel launch failed */
 };
@@ -211,6 +213,49 @@ SGMV_API int sgmv_expand(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, c
 SGMV_API int bgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
                       const sgmv_tensor* lora_idx, int64_t batches, int64_t slice_offset, int64_t slice_size,
                       int add_inputs, void* stream);
+
+/*
+ * sgmv_shrink -- the LoRA A projection whose output is the expand-slice
+ * operation's input (the page describes that input as "the low-rank
+ * intermediate activations from the LoRA A projection", I/O Contract):
+ *
+ *     out[r, n] = sum_h x^[r, h] * A[a][n, h]       for n < R, h < H
+ *
+ * for every row r of every segment b with adapter a = lora_idx[b], i.e. the
+ * expand-slice operation with lora_a in the weights' place (its N is the rank
+ * R, its K the hidden size H), the whole output row as the slice, and
+ * add_inputs off.  Same dtypes, rounding (x rounded to lora_a's dtype, fp32
+ * sums, one rounding), guards, metadata and statuses as sgmv_expand_slice.
+ *
+ *   inputs    (T_x, H)                        f16 | bf16 | f32, any strides
+ *   lora_a    (lora_num, R, H) or (lora_num, 1, R, H)   f16 | bf16, any strides
+ *   out       (T_out, R)                      f16 | bf16 | f32, contiguous; out.shape[1]
+ *             must equal R (else SGMV_ERR_OUT_WIDTH); rows outside the segments
+ *             keep their bits
+ *   workspace, workspace_bytes  optional DEVICE scratch (16-byte aligned, else
+ *             SGMV_ERR_WORKSPACE), owned by the caller and used only by the
+ *             work this call enqueues.  With it the tensor-core kernel splits
+ *             H so that every SM has work and adds the fp32 partial sums in a
+ *             second kernel, in a fixed order (deterministic); without it
+ *             (NULL or too small) each row block is one work item.  Calls
+ *             that run at the same time need separate workspaces.
+ *
+ * The tensor-core path (SGMV_VARIANT_TC) needs x and lora_a in the same half
+ * dtype with unit column stride and 16-byte aligned rows, R a multiple of 16
+ * in 16..128 and batches <= 1024; other calls run the generic kernel.
+ */
+SGMV_API int sgmv_shrink(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
+                const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+                int64_t batches, int64_t max_seq_len, void* workspace, size_t workspace_bytes, void* stream);
+
+/* sgmv_shrink_plan -- validate as sgmv_shrink does and report the variant a
+ * call with a workspace of workspace_bytes would launch, its H split count,
+ * and the workspace size (bytes) at which it would use its preferred split
+ * count (0: the call wants none).  Launches nothing. */
+SGMV_API int sgmv_shrink_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
+                     const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+                     int64_t batches, int64_t max_seq_len, size_t workspace_bytes, int* variant, int* splits,
+                     size_t* preferred_workspace_bytes);
 
 /* bgmv_plan -- validate as bgmv_expand_slice does; *variant receives the
  * kernel variant a call would launch (0 when nothing launches). */

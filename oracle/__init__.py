@@ -157,6 +157,19 @@ def bgmv_expand_slice(x, x_dt, w, w_dt, out, out_dt, lora_idx, slice_offset, sli
                         add_inputs, batches=B, nthreads=nthreads, return_pre=return_pre)
 
 
+def shrink(x, x_dt, a, a_dt, out, out_dt, seq_start, seq_len, lora_idx, batches=None, nthreads=1,
+           return_pre=False):
+    """The LoRA A projection that produces the expand input ("Implementation:
+    Predibase Lorax SGMV Expand Slice Kernel", I/O Contract, inputs):
+    out[r, n] = sum_h x[r, h] * A[a][n, h] over the rows of every segment.  It
+    is the same segmented product as expand_slice with A (lora_num, R, H) in
+    the weights' place, R output columns written from column 0, and no add."""
+    R = a.shape[-2]
+    assert out.shape[1] == R, "shrink writes whole rows: out's width must equal the rank"
+    return expand_slice(x, x_dt, a, a_dt, out, out_dt, seq_start, seq_len, lora_idx, 0, R, False,
+                        batches=batches, nthreads=nthreads, return_pre=return_pre)
+
+
 def run_problem(p, nthreads=1, return_pre=False, out=None, call=0):
     """Run the oracle on a `sgmv_inputs.Problem` (one of its slice calls)."""
     c = p.calls[call]

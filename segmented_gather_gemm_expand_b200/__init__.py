@@ -21,6 +21,8 @@ single call, which the page's Description anticipates as a fused operator.
 ``sgmv_expand`` is the standard expand the slice operation extends (the whole
 output row is the slice), and ``bgmv_expand_slice`` its fixed-length
 counterpart with one token per row (both named in the page's Description).
+``sgmv_shrink`` is the LoRA-A projection that produces the expand's input
+(I/O Contract, inputs).
 """
 import ctypes
 
@@ -28,7 +30,8 @@ import torch
 
 from . import _abi
 
-__all__ = ["sgmv_expand_slice", "sgmv_expand_multi_slice", "sgmv_expand", "bgmv_expand_slice", "plan",
+__all__ = ["sgmv_expand_slice", "sgmv_expand_multi_slice", "sgmv_expand", "bgmv_expand_slice", "sgmv_shrink",
+           "shrink_plan", "plan",
            "plan_multi_slice", "bgmv_plan", "validate_metadata", "set_variant", "device_error", "SgmvError",
            "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "VARIANT_DECODE", "library_path"]
 
@@ -133,6 +136,41 @@ def bgmv_plan(inputs, lora_b_weights, output_tensor, lora_indices_tensor, slice_
     if rc != 0:
         raise SgmvError(rc, "bgmv_plan")
     return v.value
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+
+
+def sgmv_shrink(inputs, lora_a_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor,
+                batches, max_seq_length, workspace=None):
+    """In-place SGMV shrink: ``output_tensor[r] = inputs[r] @ lora_a_weights[idx_b].T`` for the rows of
+    every segment.  ``workspace``: optional contiguous CUDA tensor of scratch (see ``shrink_plan``)."""
+    d = _args(inputs, lora_a_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor)
+    wp, wb = _ws(workspace)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_shrink(*[ctypes.byref(x) for x in d], int(batches), int(max_seq_length), wp, wb,
+                              _stream_handle(output_tensor.device))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_shrink")
+    return output_tensor
+
+
+def shrink_plan(inputs, lora_a_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor,
+                batches, max_seq_length, workspace_bytes=0):
+    """(variant, splits, preferred workspace bytes) of a shrink call with a workspace of that size."""
+    d = _args(inputs, lora_a_weights, output_tensor, b_seq_start_loc, seq_len_tensor, lora_indices_tensor)
+    v, sp, pref = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_size_t(0)
+    with torch.cuda.device(output_tensor.device):
+        rc = _lib.sgmv_shrink_plan(*[ctypes.byref(x) for x in d], int(batches), int(max_seq_length),
+                                   int(workspace_bytes), ctypes.byref(v), ctypes.byref(sp), ctypes.byref(pref))
+    if rc != 0:
+        raise SgmvError(rc, "sgmv_shrink_plan")
+    return v.value, sp.value, pref.value
 
 
 def _multi_args(inputs, lora_b_list, output_tensor, b_seq_start_loc, seq_len_tensor,

@@ -21,7 +21,7 @@ STATUS_NAMES = {
     -7: "SGMV_ERR_OUT_NOT_CONTIGUOUS", -8: "SGMV_ERR_SLICE_RANGE", -9: "SGMV_ERR_BATCHES",
     -10: "SGMV_ERR_SHAPE", -11: "SGMV_ERR_STRIDE", -12: "SGMV_ERR_TOO_LARGE",
     -13: "SGMV_ERR_VARIANT", -14: "SGMV_ERR_NUM_SLICES", -15: "SGMV_ERR_SLICE_OVERLAP",
-    -16: "SGMV_ERR_OUT_WIDTH",
+    -16: "SGMV_ERR_OUT_WIDTH", -17: "SGMV_ERR_WORKSPACE",
     -20: "SGMV_ERR_CUDA", -21: "SGMV_ERR_LAUNCH",
 }
 MAX_SLICES = 4
@@ -75,6 +75,12 @@ def load():
     lib.bgmv_expand_slice.argtypes = [P, P, P, P, i64, i64, i64, i32, vp]
     lib.bgmv_plan.restype = i32
     lib.bgmv_plan.argtypes = [P, P, P, P, i64, i64, i64, i32, ctypes.POINTER(i32)]
+    sz = ctypes.c_size_t
+    lib.sgmv_shrink.restype = i32
+    lib.sgmv_shrink.argtypes = [P, P, P, P, P, P, i64, i64, vp, sz, vp]
+    lib.sgmv_shrink_plan.restype = i32
+    lib.sgmv_shrink_plan.argtypes = [P, P, P, P, P, P, i64, i64, sz, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                     ctypes.POINTER(sz)]
     lib.sgmv_validate_metadata.restype = i32
     lib.sgmv_validate_metadata.argtypes = [P, P, P, i64, i64, i64, vp, vp]
     lib.sgmv_status_string.restype = ctypes.c_char_p

@@ -27,6 +27,7 @@ __device__ void raise_device_error(int32_t bits) { atomicOr(&g_device_error, bit
 }  // namespace sgmv
 
 #include "tc_kernel.cuh"
+#include "shrink.cuh"
 
 static_assert(SGMV_MAX_SLICES == sgmv::tc::MAX_SLICES, "one fused launch takes every slice of a call");
 
@@ -288,9 +289,96 @@ int launch_bgmv(const Call& c, cudaStream_t stream) {
     }
 }
 
+// sgmv_shrink: the expand-slice validation with lora_a in the weights' place
+// (its N is the rank, its K the hidden size) and the whole output row as the
+// slice; add_inputs is off.
+int validate_shrink(const sgmv_tensor* x, const sgmv_tensor* a, const sgmv_tensor* out, const sgmv_tensor* s,
+                    const sgmv_tensor* l, const sgmv_tensor* idx, int64_t batches, int64_t max_seq_len, Call* call) {
+    int rc;
+    if ((rc = check_basic(a))) return rc;
+    if ((rc = check_basic(out))) return rc;
+    if (a->ndim != 3 && a->ndim != 4) return SGMV_ERR_NDIM;
+    if (out->ndim != 2) return SGMV_ERR_NDIM;
+    const int64_t R = a->shape[a->ndim - 2];
+    if ((rc = validate_call(x, a, out, s, l, idx, batches, max_seq_len, 0, R, 0, call))) return rc;
+    if (out->shape[1] != R) return SGMV_ERR_OUT_WIDTH;
+    return SGMV_OK;
+}
+
+// Variant and split count of a validated, non-empty shrink call with the given workspace.
+int choose_shrink(const Call& c, const DeviceInfo& dev, int forced, const void* ws, size_t ws_bytes, int* splits) {
+    *splits = 1;
+    const bool tc_ok = dev.cc_major == 10 && shr::supports(c.p);
+    int v;
+    if (forced == SGMV_VARIANT_SIMT) v = SGMV_VARIANT_SIMT;
+    else if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;
+    else if (forced == SGMV_VARIANT_TC) v = tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
+    else v = tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
+    if (v == SGMV_VARIANT_TC && ws) {
+        int sp = shr::preferred_splits(c.p, dev.sm_count);
+        while (sp > 1 && (size_t)shr::workspace_bytes_for(c.p, sp) > ws_bytes) sp /= 2;
+        *splits = sp;
+    }
+    return v;
+}
+
+int launch_shrink(const Call& c, const DeviceInfo& dev, int splits, float* ws, cudaStream_t stream) {
+    shr::Plan pl;
+    if (!shr::make_plan(c.p, dev.sm_count, splits, tc::encode_fn(), &pl)) return SGMV_ERR_VARIANT;
+    switch (c.p.out_dt) {
+        case SGMV_F32: return shr::launch_dt<SGMV_F32>(pl, c.p, ws, stream);
+        case SGMV_BF16: return shr::launch_dt<SGMV_BF16>(pl, c.p, ws, stream);
+        default: return shr::launch_dt<SGMV_F16>(pl, c.p, ws, stream);
+    }
+}
+
 }  // namespace
 
 extern "C" {
+
+int sgmv_shrink(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
+                const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+                int64_t batches, int64_t max_seq_len, void* workspace, size_t workspace_bytes, void* stream) {
+    Call c;
+    int rc = validate_shrink(inputs, lora_a, out, seq_start, seq_len, lora_idx, batches, max_seq_len, &c);
+    if (rc) return rc;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 15)) return SGMV_ERR_WORKSPACE;
+    if (c.empty) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    int splits = 1;
+    const int v = choose_shrink(c, dev, g_forced_variant.load(), workspace, workspace_bytes, &splits);
+    if (v < 0) return v;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (v == SGMV_VARIANT_TC) return launch_shrink(c, dev, splits, static_cast<float*>(workspace), st);
+    return launch_simt(c, dev, st);
+}
+
+int sgmv_shrink_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
+                     const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
+                     int64_t batches, int64_t max_seq_len, size_t workspace_bytes, int* variant, int* splits,
+                     size_t* preferred_workspace_bytes) {
+    if (!variant || !splits || !preferred_workspace_bytes) return SGMV_ERR_NULL_ARG;
+    *variant = 0;
+    *splits = 0;
+    *preferred_workspace_bytes = 0;
+    Call c;
+    int rc = validate_shrink(inputs, lora_a, out, seq_start, seq_len, lora_idx, batches, max_seq_len, &c);
+    if (rc) return rc;
+    if (c.empty) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    int sp = 1;
+    static const char dummy = 0;   // a non-null stand-in: only the size matters here
+    const int v = choose_shrink(c, dev, g_forced_variant.load(), workspace_bytes ? &dummy : nullptr, workspace_bytes,
+                                &sp);
+    if (v < 0) return v;
+    *variant = v;
+    *splits = v == SGMV_VARIANT_TC ? sp : 1;
+    if (v == SGMV_VARIANT_TC)
+        *preferred_workspace_bytes = (size_t)shr::workspace_bytes_for(c.p, shr::preferred_splits(c.p, dev.sm_count));
+    return SGMV_OK;
+}
 
 int sgmv_expand(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, const sgmv_tensor* out,
                 const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
@@ -478,7 +566,8 @@ const char* sgmv_status_string(int code) {
         case SGMV_ERR_VARIANT: return "the forced kernel variant cannot run this call";
         case SGMV_ERR_NUM_SLICES: return "num_slices outside [1, SGMV_MAX_SLICES]";
         case SGMV_ERR_SLICE_OVERLAP: return "two slices of a multi-slice call overlap";
-        case SGMV_ERR_OUT_WIDTH: return "sgmv_expand: out.shape[1] != lora_b.shape[-2]";
+        case SGMV_ERR_OUT_WIDTH: return "out.shape[1] != lora_b.shape[-2] (plain expand and shrink write whole rows)";
+        case SGMV_ERR_WORKSPACE: return "workspace is not 16-byte aligned";
         case SGMV_ERR_CUDA: return "a CUDA runtime call failed";
         case SGMV_ERR_LAUNCH: return "kernel launch failed";
         default: return "unknown status";

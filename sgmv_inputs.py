@@ -79,6 +79,7 @@ class Problem:
     calls: List[SliceCall]
     meta_dt: str = "int64"   # dtype the metadata is handed to the library in
     seed: int = 0
+    op: str = "slice"        # "slice": sgmv_expand_slice; "bgmv": one token per row (starts b, lengths 1)
 
     @property
     def batches(self) -> int:
@@ -187,12 +188,28 @@ def decode_mix(seed: int = 0) -> Problem:
                    lengths, idx, True, [SliceCall(w, 5120, N)], seed=seed)
 
 
+def decode_bgmv(seed: int = 0) -> Problem:
+    """The decode step of the decode-like mix: one token per sequence (the BGMV
+    case), 256 sequences with distinct adapters out of 256, 10% at -1."""
+    rng = np.random.default_rng(seed)
+    B, K, A, N = 256, 32, 256, 5120
+    lengths = np.ones(B, dtype=np.int64)
+    idx = rng.permutation(A)[:B].astype(np.int64)
+    idx[_minus_one_mask(rng, B, 0.10)] = -1
+    x = normal(rng, (B, K), 1.0, "bf16")
+    w = normal(rng, (A, N, K), 0.02, "bf16")
+    y0 = normal(rng, (B, 3 * N), 1.0, "bf16")
+    return Problem("decode_bgmv", x, "bf16", "bf16", y0, "bf16", exclusive_cumsum(lengths),
+                   lengths, idx, True, [SliceCall(w, 5120, N)], seed=seed, op="bgmv")
+
+
 WORKLOADS = {
     "tiny": tiny,
     "qkv_prefill": qkv_prefill,
     "mlp_mixed": mlp_mixed,
     "long_single": long_single,
     "decode_mix": decode_mix,
+    "decode_bgmv": decode_bgmv,
 }
 
 

@@ -272,3 +272,55 @@ def test_decode_variant_is_only_for_bgmv():
         assert call(a) == _abi.STATUS["SGMV_ERR_VARIANT"]
     finally:
         lib.sgmv_set_variant(prev)
+
+
+# ------------------------------------------------------------ shrink
+
+def shrink_args(**over):
+    T, H, A, R, B = 20, 256, 3, 16, 4
+    a = dict(
+        x=_abi.make_tensor(FAKE, _abi.BF16, (T, H), (H, 1)),
+        w=_abi.make_tensor(FAKE, _abi.BF16, (A, R, H), (R * H, H, 1)),
+        out=_abi.make_tensor(FAKE, _abi.F32, (T, R), (R, 1)),
+        s=_abi.make_tensor(FAKE, _abi.I64, (B,), (1,)),
+        l=_abi.make_tensor(FAKE, _abi.I64, (B,), (1,)),
+        i=_abi.make_tensor(FAKE, _abi.I32, (B,), (1,)),
+        batches=B, max_seq_len=7, ws=None, ws_bytes=0,
+    )
+    a.update(over)
+    return a
+
+
+def shrink_call(a):
+    lib = _abi.load()
+    r = ctypes.byref
+    return lib.sgmv_shrink(r(a["x"]), r(a["w"]), r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]), a["batches"],
+                           a["max_seq_len"], a["ws"], a["ws_bytes"], None)
+
+
+SHRINK_BAD = {
+    "out_width_not_rank": (dict(out=_abi.make_tensor(FAKE, _abi.F32, (20, 32), (32, 1))), "SGMV_ERR_OUT_WIDTH"),
+    "hidden_size_mismatch": (dict(x=_abi.make_tensor(FAKE, _abi.BF16, (20, 128), (128, 1))), "SGMV_ERR_RANK_MISMATCH"),
+    "a_2d": (dict(w=_abi.make_tensor(FAKE, _abi.BF16, (16, 256), (256, 1))), "SGMV_ERR_NDIM"),
+    "a_f32": (dict(w=_abi.make_tensor(FAKE, _abi.F32, (3, 16, 256), (16 * 256, 256, 1))), "SGMV_ERR_DTYPE"),
+    "a_4d_bad_unit_dim": (dict(w=_abi.make_tensor(FAKE, _abi.BF16, (3, 2, 16, 256), (2 * 16 * 256, 16 * 256, 256, 1))),
+                          "SGMV_ERR_LAYOUT_4D"),
+    "out_not_contiguous": (dict(out=_abi.make_tensor(FAKE, _abi.F32, (20, 16), (17, 1))), "SGMV_ERR_OUT_NOT_CONTIGUOUS"),
+    "meta_short": (dict(batches=6), "SGMV_ERR_BATCHES"),
+    "misaligned_workspace": (dict(ws=FAKE + 4, ws_bytes=1 << 20), "SGMV_ERR_WORKSPACE"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SHRINK_BAD))
+def test_shrink_invalid_arguments_fail_before_launch(case):
+    over, code = SHRINK_BAD[case]
+    assert shrink_call(shrink_args(**over)) == _abi.STATUS[code]
+
+
+def test_shrink_plan_null_outputs():
+    lib = _abi.load()
+    a = shrink_args()
+    r = ctypes.byref
+    v = ctypes.c_int(0)
+    assert lib.sgmv_shrink_plan(r(a["x"]), r(a["w"]), r(a["out"]), r(a["s"]), r(a["l"]), r(a["i"]), 4, 7, 0,
+                                r(v), None, None) == _abi.STATUS["SGMV_ERR_NULL_ARG"]

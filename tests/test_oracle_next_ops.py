@@ -120,3 +120,54 @@ def test_plain_expand_requires_whole_rows():
     c = p.calls[0]
     with pytest.raises(AssertionError):
         oracle.expand(p.x, p.x_dt, c.w, p.w_dt, p.y0, p.out_dt, p.seq_start, p.seq_len, p.lora_idx, True)
+
+
+# ------------------------------------------------------------------ shrink
+
+def shrink_problem(seed, lengths, H, R, A, **kw):
+    """x (T, H), lora_a (A, R, H) in calls[0].w, out (T, R)."""
+    return gen.custom(seed=seed, lengths=lengths, K=H, N=R, H=R, offset=0, num_adapters=A, add_inputs=False, **kw)
+
+
+@pytest.mark.parametrize("x_dt,a_dt,out_dt", [("bf16", "bf16", "f32"), ("f16", "f16", "bf16"), ("f32", "bf16", "f16")])
+def test_shrink_matches_dense_per_adapter(x_dt, a_dt, out_dt):
+    p = shrink_problem(11, [7, 0, 20, 3], H=300, R=16, A=3, idx=[2, 1, 0, -1], x_dt=x_dt, w_dt=a_dt, out_dt=out_dt)
+    c = p.calls[0]
+    out, pre = oracle.shrink(p.x, p.x_dt, c.w, p.w_dt, p.y0, p.out_dt, p.seq_start, p.seq_len, p.lora_idx,
+                             return_pre=True)
+    ra = np.full(p.y0.shape[0], -1)
+    for s, L, a in zip(p.seq_start, p.seq_len, p.lora_idx):
+        if a >= 0:
+            ra[s:s + L] = a
+    want = dense_rows(p.x, p.x_dt, c.w, p.w_dt, p.y0, p.out_dt, ra, 0, False)
+    written = ra >= 0
+    np.testing.assert_allclose(pre[written], want[written], rtol=1e-12, atol=1e-12)
+    check_rounded(out, want, written, 0, 16, out_dt, p.y0)
+
+
+def test_shrink_integer_inputs_are_exact():
+    p = shrink_problem(12, [5, 9], H=64, R=32, A=2, idx=[1, 0], integer=True, out_dt="f32")
+    c = p.calls[0]
+    out = oracle.shrink(p.x, p.x_dt, c.w, p.w_dt, p.y0, p.out_dt, p.seq_start, p.seq_len, p.lora_idx)
+    xi = indep_decode(p.x, p.x_dt).astype(np.int64)
+    ai = indep_decode(c.w, p.w_dt).astype(np.int64)
+    for s, L, a in zip(p.seq_start, p.seq_len, p.lora_idx):
+        exact = xi[s:s + L] @ ai[a].T
+        assert np.array_equal(out[s:s + L].astype(np.float64), exact.astype(np.float64))
+
+
+def test_shrink_then_expand_is_the_lora_delta():
+    """Shrink into an fp32 intermediate, then expand: the slice gets x . A^T . B^T (the LoRA update)."""
+    H, R, N, A = 96, 16, 40, 2
+    p = shrink_problem(13, [6, 4], H=H, R=R, A=A, idx=[1, 0], out_dt="f32", y_scale=0.0)
+    a = p.calls[0].w
+    mid = oracle.shrink(p.x, p.x_dt, a, p.w_dt, p.y0, "f32", p.seq_start, p.seq_len, p.lora_idx)
+    rng = np.random.default_rng(3)
+    b = gen.normal(rng, (A, N, R), 0.02, "bf16")
+    y0 = np.zeros((10, N), np.float32)
+    y = oracle.expand(mid, "f32", b, "bf16", y0, "f32", p.seq_start, p.seq_len, p.lora_idx, False)
+    xd = indep_decode(p.x, p.x_dt)
+    for s, L, ai in zip(p.seq_start, p.seq_len, p.lora_idx):
+        delta = xd[s:s + L] @ indep_decode(a[ai], "bf16").T
+        delta = indep_cast(delta.astype(np.float32).astype(np.float64), "bf16") @ indep_decode(b[ai], "bf16").T
+        np.testing.assert_allclose(y[s:s + L], delta, rtol=1e-5, atol=1e-6)

@@ -93,6 +93,7 @@ enum {
     SGMV_ERR_SLICE_OVERLAP = -15,    /* two non-empty slices of one call share a column */
     SGMV_ERR_OUT_WIDTH = -16,        /* sgmv_expand / sgmv_shrink: out.shape[1] != lora_b/lora_a.shape[-2] */
     SGMV_ERR_WORKSPACE = -17,        /* sgmv_shrink: workspace not 16-byte aligned */
+    SGMV_ERR_SCRATCH = -18,          /* sgmv_shrink_static_scratch: the call needs more than the static scratch */
     SGMV_ERR_CUDA = -20,             /* a CUDA runtime call failed */
     SGMV_ERR_LAUNCH = -21            /* a kernel launch failed */
 };
@@ -247,6 +248,43 @@ SGMV_API int bgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lor
 SGMV_API int sgmv_shrink(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
                 const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
                 int64_t batches, int64_t max_seq_len, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device scratch that sgmv_shrink_static_scratch owns on every device. */
+#define SGMV_SHRINK_STATIC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * sgmv_shrink_static_scratch -- sgmv_shrink for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this entry point exists for
+ * the caller, not for the method.
+ *
+ * Some callers are not allowed to allocate: a runtime that reserves all of
+ * the GPU's memory when it starts and then forbids further allocations, a
+ * plugin host that hands its plugins only their input and output buffers, or
+ * a serving loop that must never stall on cudaMalloc, which can synchronise
+ * the device.  Such a caller cannot provide sgmv_shrink's workspace, and
+ * without one the shrink runs with one work item per row block.  This entry
+ * point instead keeps the partial sums in a scratch array that the library
+ * itself declares as a file-scope device variable of
+ * SGMV_SHRINK_STATIC_SCRATCH_BYTES, which every GPU that loads the library
+ * holds until the process exits.  It computes exactly what sgmv_shrink
+ * computes with a workspace that fits its preferred split count, and takes the
+ * same arguments without the workspace.
+ *
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and keeps it; make that first call before any
+ *     stream capture.  Later calls only read the kept address.
+ *   - It allocates nothing and calls no allocating routine.
+ *   - A call whose partial sums need more than SGMV_SHRINK_STATIC_SCRATCH_BYTES
+ *     (splits x min(T_x, T_out) x R x 4 bytes) returns SGMV_ERR_SCRATCH before
+ *     anything is enqueued; sgmv_shrink with a workspace of your own takes it.
+ *   - Every call on a device shares the one array, and it keeps whatever the
+ *     last call left there: each call writes every partial sum before it reads
+ *     it, so nothing needs to start at zero, but two calls whose work overlaps
+ *     on the GPU (different streams, no ordering between them) race on it.
+ */
+SGMV_API int sgmv_shrink_static_scratch(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
+                               const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                               const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len, void* stream);
 
 /* sgmv_shrink_plan -- validate as sgmv_shrink does and report the variant a
  * call with a workspace of workspace_bytes would launch, its H split count,

@@ -22,6 +22,7 @@ STATUS_NAMES = {
     -10: "SGMV_ERR_SHAPE", -11: "SGMV_ERR_STRIDE", -12: "SGMV_ERR_TOO_LARGE",
     -13: "SGMV_ERR_VARIANT", -14: "SGMV_ERR_NUM_SLICES", -15: "SGMV_ERR_SLICE_OVERLAP",
     -16: "SGMV_ERR_OUT_WIDTH", -17: "SGMV_ERR_WORKSPACE",
+    -18: "SGMV_ERR_SCRATCH",
     -20: "SGMV_ERR_CUDA", -21: "SGMV_ERR_LAUNCH",
 }
 MAX_SLICES = 4
@@ -78,6 +79,8 @@ def load():
     sz = ctypes.c_size_t
     lib.sgmv_shrink.restype = i32
     lib.sgmv_shrink.argtypes = [P, P, P, P, P, P, i64, i64, vp, sz, vp]
+    lib.sgmv_shrink_static_scratch.restype = i32
+    lib.sgmv_shrink_static_scratch.argtypes = [P, P, P, P, P, P, i64, i64, vp]
     lib.sgmv_shrink_plan.restype = i32
     lib.sgmv_shrink_plan.argtypes = [P, P, P, P, P, P, i64, i64, sz, ctypes.POINTER(i32), ctypes.POINTER(i32),
                                      ctypes.POINTER(sz)]

@@ -354,6 +354,70 @@ int sgmv_shrink(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv
     return launch_simt(c, dev, st);
 }
 
+}  // extern "C"
+
+// Scratch of sgmv_shrink_static_scratch: the partial sums of split-H shrinks
+// for callers that cannot allocate.  In host code this name is only a
+// stand-in for the device variable: its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) float g_shrink_scratch[SGMV_SHRINK_STATIC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+float* g_shrink_scratch_ptr[kMaxDevices];
+std::mutex g_shrink_scratch_mu;
+
+// Device address of g_shrink_scratch on the current device (looked up on the
+// first call there), or nullptr with *rc set.
+float* static_scratch(int* rc) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *rc = SGMV_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_shrink_scratch_mu);
+    if (!g_shrink_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_shrink_scratch) != cudaSuccess || !ptr) {
+            *rc = SGMV_ERR_CUDA;
+            return nullptr;
+        }
+        g_shrink_scratch_ptr[dev] = static_cast<float*>(ptr);
+    }
+    *rc = SGMV_OK;
+    return g_shrink_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int sgmv_shrink_static_scratch(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
+                               const sgmv_tensor* seq_start, const sgmv_tensor* seq_len,
+                               const sgmv_tensor* lora_idx, int64_t batches, int64_t max_seq_len, void* stream) {
+    Call c;
+    int rc = validate_shrink(inputs, lora_a, out, seq_start, seq_len, lora_idx, batches, max_seq_len, &c);
+    if (rc) return rc;
+    if (c.empty) return SGMV_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev))) return rc;
+    const int forced = g_forced_variant.load();
+    int splits = 1;
+    // the split count sgmv_shrink would use with an unlimited workspace
+    const int v0 = choose_shrink(c, dev, forced, nullptr, 0, &splits);
+    if (v0 < 0) return v0;
+    if (v0 == SGMV_VARIANT_TC) {
+        splits = shr::preferred_splits(c.p, dev.sm_count);
+        if ((uint64_t)shr::workspace_bytes_for(c.p, splits) > (uint64_t)SGMV_SHRINK_STATIC_SCRATCH_BYTES)
+            return SGMV_ERR_SCRATCH;
+    }
+    float* scratch = static_scratch(&rc);
+    if (!scratch) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (v0 == SGMV_VARIANT_TC) return launch_shrink(c, dev, splits, scratch, st);
+    return launch_simt(c, dev, st);
+}
+
 int sgmv_shrink_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const sgmv_tensor* out,
                      const sgmv_tensor* seq_start, const sgmv_tensor* seq_len, const sgmv_tensor* lora_idx,
                      int64_t batches, int64_t max_seq_len, size_t workspace_bytes, int* variant, int* splits,
@@ -568,6 +632,7 @@ const char* sgmv_status_string(int code) {
         case SGMV_ERR_SLICE_OVERLAP: return "two slices of a multi-slice call overlap";
         case SGMV_ERR_OUT_WIDTH: return "out.shape[1] != lora_b.shape[-2] (plain expand and shrink write whole rows)";
         case SGMV_ERR_WORKSPACE: return "workspace is not 16-byte aligned";
+        case SGMV_ERR_SCRATCH: return "the call needs more scratch than sgmv_shrink_static_scratch's static array holds";
         case SGMV_ERR_CUDA: return "a CUDA runtime call failed";
         case SGMV_ERR_LAUNCH: return "kernel launch failed";
         default: return "unknown status";

@@ -53,6 +53,8 @@ WORKLOAD_TEXT = {
     "tiny": "tiny: 4 seqs [4,6,3,7], rank 16, fp16, slice 128 at 128, overwrite",
     "decode_bgmv": "decode step (bgmv_expand_slice): 256 one-token rows, 256 distinct adapters (10% -1), "
                    "rank 32, bf16, slice 5120 at 5120 of 256 x 15360, add_inputs",
+    "qkv_shrink": "LoRA-A shrink feeding the QKV prefill (sgmv_shrink): 16 seqs U[64,1024], 32 adapters "
+                  "(10% -1), hidden 4096 -> rank 16, bf16, split-H workspace",
 }
 
 DT_SIZE = {"f16": 2, "bf16": 2, "f32": 4}
@@ -187,10 +189,12 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- runtime helpers
 
-def make_calls(p, dev_tensors, sg_abi, stream_handle_fn):
+def make_calls(p, dev_tensors, sg_abi, stream_handle_fn, workspace=None):
     """Pre-marshalled C-ABI argument tuples, one per slice call."""
     import segmented_gather_gemm_expand_b200 as sg
     x, ws, y, meta = dev_tensors
+    wsp = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+    wsb = workspace.numel() if workspace is not None else 0
     descs = []
     for c, call in enumerate(p.calls):
         d = [sg._desc(t) for t in (x, ws[c], y, *meta)]
@@ -199,7 +203,10 @@ def make_calls(p, dev_tensors, sg_abi, stream_handle_fn):
 
     def run(c, stream):
         d, off, size = descs[c]
-        if p.op == "bgmv":   # x, B, out and lora_idx only: row b is one token
+        if p.op == "shrink":
+            rc = lib.sgmv_shrink(*[ctypes.byref(t) for t in d], p.batches, p.max_seq_len, wsp, wsb,
+                                 ctypes.c_void_p(stream))
+        elif p.op == "bgmv":   # x, B, out and lora_idx only: row b is one token
             rc = lib.bgmv_expand_slice(ctypes.byref(d[0]), ctypes.byref(d[1]), ctypes.byref(d[2]),
                                        ctypes.byref(d[5]), p.batches, off, size, int(p.add_inputs),
                                        ctypes.c_void_p(stream))
@@ -207,7 +214,7 @@ def make_calls(p, dev_tensors, sg_abi, stream_handle_fn):
             rc = lib.sgmv_expand_slice(*[ctypes.byref(t) for t in d], p.batches, p.max_seq_len, off, size,
                                        int(p.add_inputs), ctypes.c_void_p(stream))
         if rc != 0:
-            raise sg.SgmvError(rc, "bgmv_expand_slice" if p.op == "bgmv" else "sgmv_expand_slice")
+            raise sg.SgmvError(rc, {"bgmv": "bgmv_expand_slice", "shrink": "sgmv_shrink"}.get(p.op, "sgmv_expand_slice"))
     return run, descs
 
 
@@ -290,15 +297,25 @@ def bench_ours(args, rank, world, device):
     ws = [w.to(device) for w in hws]
     y = hy.to(device)
     meta = [m.to(device) for m in hmeta]
-    run, _ = make_calls(p, (x, ws, y, meta), _abi, None)
+    workspace = None
+    if p.op == "shrink":
+        _, _, pref = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, 1 << 34)
+        workspace = torch.empty(max(pref, 16), dtype=torch.uint8, device=device)
+    run, _ = make_calls(p, (x, ws, y, meta), _abi, None, workspace=workspace)
     ncalls = len(p.calls)
-    if p.op == "bgmv":
+    shrink_splits = 0
+    if p.op == "shrink":
+        v_used, shrink_splits, _ = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len,
+                                                  workspace.numel())
+    elif p.op == "bgmv":
         v_used = sg.bgmv_plan(x, ws[0], y, meta[2], p.calls[0].slice_offset, p.calls[0].slice_size,
                               p.add_inputs)
     else:
         v_used = sg.plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, p.calls[0].slice_offset,
                          p.calls[0].slice_size, p.add_inputs)
     variant_name = {1: "simt", 2: "tc", 3: "decode"}.get(v_used, str(v_used))
+    # kernel launches one call makes (a split shrink adds the partial-sum reduction)
+    launches_per_call = 2 if (p.op == "shrink" and shrink_splits > 1) else 1
 
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
@@ -449,11 +466,13 @@ def bench_ours(args, rank, world, device):
                      "frac": achieved / peak, "traffic": recorded_traffic(args.workload, variant_name),
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6650 GB/s",
-                     "kernel": f"sgmv expand-slice ({variant_name})",
+                     "kernel": f"{ {'bgmv': 'bgmv_expand_slice', 'shrink': 'sgmv_shrink'}.get(p.op, 'sgmv_expand_slice') } "
+                               f"({variant_name}{', %d H splits + reduction' % shrink_splits if shrink_splits > 1 else ''})",
                      "launch_ms_avg": avg_launch_ms, "bytes_per_launch": call_bytes,
                      "launches_timed": K * ncalls,
-                     "launch_ms_note": "timed region / launches (back-to-back launches, gaps included)"},
-        "gpu_launches": K * ncalls,
+                     "launch_ms_note": "timed region / calls (back-to-back calls, gaps included; a split shrink "
+                                       "call is its main kernel plus the reduction)"},
+        "gpu_launches": K * ncalls * launches_per_call,
         "clocks": clocks,
         "fused_multi_slice": fused,
         "e2e": e2e,

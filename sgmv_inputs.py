@@ -79,7 +79,8 @@ class Problem:
     calls: List[SliceCall]
     meta_dt: str = "int64"   # dtype the metadata is handed to the library in
     seed: int = 0
-    op: str = "slice"        # "slice": sgmv_expand_slice; "bgmv": one token per row (starts b, lengths 1)
+    op: str = "slice"        # "slice": sgmv_expand_slice; "bgmv": one token per row (starts b, lengths 1);
+                             # "shrink": sgmv_shrink (x is (T, H), calls[0].w is lora_a (A, R, H), out (T, R))
 
     @property
     def batches(self) -> int:
@@ -203,6 +204,23 @@ def decode_bgmv(seed: int = 0) -> Problem:
                    lengths, idx, True, [SliceCall(w, 5120, N)], seed=seed, op="bgmv")
 
 
+def qkv_shrink(seed: int = 0) -> Problem:
+    """The LoRA-A step that feeds the fused-QKV prefill batch: the same 16
+    sequences (lengths U[64,1024], 10% at -1, 32 adapters), hidden size 4096
+    projected to rank 16, bf16 in and out."""
+    rng = np.random.default_rng(seed)
+    B, R, A, H = 16, 16, 32, 4096
+    lengths = rng.integers(64, 1024 + 1, size=B).astype(np.int64)
+    idx = rng.integers(0, A, size=B).astype(np.int64)
+    idx[_minus_one_mask(rng, B, 0.10)] = -1
+    T = int(lengths.sum())
+    x = normal(rng, (T, H), 1.0, "bf16")
+    a = normal(rng, (A, R, H), 0.02, "bf16")
+    y0 = normal(rng, (T, R), 1.0, "bf16")
+    return Problem("qkv_shrink", x, "bf16", "bf16", y0, "bf16", exclusive_cumsum(lengths), lengths, idx, False,
+                   [SliceCall(a, 0, R)], seed=seed, op="shrink")
+
+
 WORKLOADS = {
     "tiny": tiny,
     "qkv_prefill": qkv_prefill,
@@ -210,6 +228,7 @@ WORKLOADS = {
     "long_single": long_single,
     "decode_mix": decode_mix,
     "decode_bgmv": decode_bgmv,
+    "qkv_shrink": qkv_shrink,
 }
 
 

@@ -103,7 +103,9 @@ enum {
     SGMV_VARIANT_AUTO = 0,
     SGMV_VARIANT_SIMT = 1,   /* generic CUDA-core kernel: any strides, rank, alignment */
     SGMV_VARIANT_TC = 2,     /* tcgen05 tensor-core kernel with TMA staging */
-    SGMV_VARIANT_DECODE = 3  /* bgmv_expand_slice's one-token-per-row kernel (vector loads) */
+    SGMV_VARIANT_DECODE = 3, /* bgmv_expand_slice's one-token-per-row kernel (vector loads) */
+    SGMV_VARIANT_TC_WIDE = 4 /* the tensor-core kernel with 256-column n-tiles forced (tests); plans report
+                                SGMV_VARIANT_TC.  SGMV_VARIANT_TC and AUTO let the library pick 128 or 256 */
 };
 
 /*

@@ -33,10 +33,11 @@ from . import _abi
 __all__ = ["sgmv_expand_slice", "sgmv_expand_multi_slice", "sgmv_expand", "bgmv_expand_slice", "sgmv_shrink",
            "shrink_plan", "plan",
            "plan_multi_slice", "bgmv_plan", "validate_metadata", "set_variant", "device_error", "SgmvError",
-           "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "VARIANT_DECODE", "library_path"]
+           "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC", "VARIANT_DECODE", "VARIANT_TC_WIDE", "library_path"]
 
 VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC = _abi.VARIANT_AUTO, _abi.VARIANT_SIMT, _abi.VARIANT_TC
 VARIANT_DECODE = _abi.VARIANT_DECODE
+VARIANT_TC_WIDE = _abi.VARIANT_TC_WIDE
 library_path = _abi.LIB_PATH
 
 _DTYPES = {torch.float16: _abi.F16, torch.bfloat16: _abi.BF16, torch.float32: _abi.F32,

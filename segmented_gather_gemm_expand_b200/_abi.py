@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(HERE, "libsgmv.so")
 F16, BF16, F32, I32, I64 = 0, 1, 2, 3, 4
 
 SGMV_OK = 0
-VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC, VARIANT_DECODE = 0, 1, 2, 3
+VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC, VARIANT_DECODE, VARIANT_TC_WIDE = 0, 1, 2, 3, 4
 
 STATUS_NAMES = {
     0: "SGMV_OK", -1: "SGMV_ERR_NULL_ARG", -2: "SGMV_ERR_DTYPE", -3: "SGMV_ERR_NDIM",

@@ -5,9 +5,15 @@
 // there is no B tile to reuse across rows, so nothing is staged: every thread
 // streams the two B rows of its two output columns with 16-byte loads
 // (consecutive threads read consecutive rows, so a warp reads one contiguous
-// stretch of B), x's row is rounded to the weights' dtype into shared memory
-// once per row, products are summed in fp32 in k order, and the result (plus
-// the old value in add mode) is rounded once.
+// stretch of B).  A row's loads -- its B rows, its x row and, in add mode, the
+// old output -- are all issued before the first of them is used, so a row
+// costs one memory round trip per 32 ranks, and the register budget leaves
+// room for eight CTAs per SM, so enough loads are in flight to cover DRAM
+// latency.  When x is already in B's dtype
+// each thread reads x's row directly (16-byte loads, served from L1); other x
+// dtypes are rounded to B's dtype once per row into shared memory.  Products
+// are summed in fp32 in k order and the result (plus the old value in add
+// mode) is rounded once.
 //
 // Grid: x = 256-column tile of the slice, y = rows (grid-stride).
 #pragma once
@@ -19,6 +25,8 @@ namespace sgmv {
 constexpr int BGMV_THREADS = 128;
 constexpr int BGMV_COLS = 2 * BGMV_THREADS;   // columns per CTA
 constexpr int BGMV_MAX_K = 256;
+constexpr int BGMV_KC = 32;                   // ranks per round trip
+constexpr int BGMV_MIN_CTAS = 8;              // CTAs per SM the register budget must allow
 
 // Element e (0..7) of 8 packed 16-bit values as a float.
 __device__ __forceinline__ float half8_elem(const uint4& v, int e, bool bf16) {
@@ -27,8 +35,9 @@ __device__ __forceinline__ float half8_elem(const uint4& v, int e, bool bf16) {
     return bf16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
 }
 
-template <int OUT_DT, bool ADD>
-__global__ void __launch_bounds__(BGMV_THREADS)
+// XVEC: x has B's dtype, unit column stride and 16-byte aligned rows.
+template <int OUT_DT, bool ADD, bool XVEC>
+__global__ void __launch_bounds__(BGMV_THREADS, BGMV_MIN_CTAS)
 bgmv_expand_kernel(Problem p) {
     __shared__ float sx[BGMV_MAX_K];
     const int tid = threadIdx.x;
@@ -36,37 +45,55 @@ bgmv_expand_kernel(Problem p) {
     const int64_t n = (int64_t)blockIdx.x * BGMV_COLS + 2 * tid;   // first of this thread's two columns
     const int64_t lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int K = (int)p.K;
+    const bool mine = n < p.N;
+    const bool two = n + 1 < p.N;
 
     for (int64_t b = blockIdx.y; b < p.batches; b += gridDim.y) {
         const int64_t a = load_meta(p.idx, b);
         if (a < 0 || a >= p.lora_num || b >= lim) continue;     // uniform across the CTA
-        __syncthreads();   // the previous row's sx is no longer read
-        for (int k = tid; k < K; k += BGMV_THREADS)
-            sx[k] = round_to(load_elem(p.x, p.x_dt, b * p.x_rs + k * p.x_cs), p.w_dt);
-        __syncthreads();
-        if (n >= p.N) continue;
-        const bool two = n + 1 < p.N;
+        const int64_t oi = b * p.H + p.off + n;
+        float old0 = 0.f, old1 = 0.f;
+        if (ADD && mine) {
+            old0 = load_elem(p.out, OUT_DT, oi);
+            if (two) old1 = load_elem(p.out, OUT_DT, oi + 1);
+        }
+        if (!XVEC) {
+            __syncthreads();   // the previous row's sx is no longer read
+            for (int k = tid; k < K; k += BGMV_THREADS)
+                sx[k] = round_to(load_elem(p.x, p.x_dt, b * p.x_rs + k * p.x_cs), p.w_dt);
+            __syncthreads();
+        }
+        if (!mine) continue;
         const uint4* w0 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.w) + a * p.w_as + n * p.w_ns);
         const uint4* w1 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.w) + a * p.w_as +
                                                          (two ? n + 1 : n) * p.w_ns);
+        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + b * p.x_rs);
         float acc0 = 0.f, acc1 = 0.f;
-        for (int k8 = 0; k8 < K / 8; ++k8) {
-            const uint4 v0 = __ldg(w0 + k8);
-            const uint4 v1 = __ldg(w1 + k8);
+        for (int k0 = 0; k0 < K; k0 += BGMV_KC) {
+            const int kn = min(BGMV_KC, K - k0) / 8;   // 16-byte pieces in this round trip
+            uint4 v0[BGMV_KC / 8], v1[BGMV_KC / 8], vx[BGMV_KC / 8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float xv = sx[k8 * 8 + e];
-                acc0 = fmaf(xv, half8_elem(v0, e, w_bf16), acc0);
-                acc1 = fmaf(xv, half8_elem(v1, e, w_bf16), acc1);
+            for (int j = 0; j < BGMV_KC / 8; ++j) {
+                if (j < kn) {
+                    v0[j] = __ldg(w0 + k0 / 8 + j);
+                    v1[j] = __ldg(w1 + k0 / 8 + j);
+                    if (XVEC) vx[j] = __ldg(xr + k0 / 8 + j);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < BGMV_KC / 8; ++j) {
+                if (j < kn) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float xv = XVEC ? half8_elem(vx[j], e, w_bf16) : sx[k0 + j * 8 + e];
+                        acc0 = fmaf(xv, half8_elem(v0[j], e, w_bf16), acc0);
+                        acc1 = fmaf(xv, half8_elem(v1[j], e, w_bf16), acc1);
+                    }
+                }
             }
         }
-        const int64_t oi = b * p.H + p.off + n;
-        if (ADD) {
-            acc0 += load_elem(p.out, OUT_DT, oi);
-            if (two) acc1 += load_elem(p.out, OUT_DT, oi + 1);
-        }
-        store_elem(p.out, OUT_DT, oi, acc0);
-        if (two) store_elem(p.out, OUT_DT, oi + 1, acc1);
+        store_elem(p.out, OUT_DT, oi, ADD ? old0 + acc0 : acc0);
+        if (two) store_elem(p.out, OUT_DT, oi + 1, ADD ? old1 + acc1 : acc1);
     }
 }
 

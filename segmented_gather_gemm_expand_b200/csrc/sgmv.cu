@@ -187,12 +187,16 @@ int launch_simt(const Call& c, const DeviceInfo& dev, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? SGMV_OK : SGMV_ERR_LAUNCH;
 }
 
+// n-tile width a forced variant fixes for the tensor-core kernel (0: the library chooses).
+int forced_bn(int forced) { return forced == SGMV_VARIANT_TC_WIDE ? 256 : 0; }
+
 // Which variant runs a validated, non-empty call.
 int choose_variant(const Call& c, const DeviceInfo& dev, int forced) {
-    const bool tc_ok = dev.cc_major == 10 && tc_supports(&c.p, 1);
+    const bool tc_ok = dev.cc_major == 10 && tc_supports(&c.p, 1, forced_bn(forced));
     if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
     if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;   // bgmv_expand_slice's kernel only
-    if (forced == SGMV_VARIANT_TC) return tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
+    if (forced == SGMV_VARIANT_TC || forced == SGMV_VARIANT_TC_WIDE)
+        return tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
     return tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
 }
 
@@ -231,7 +235,7 @@ int choose_multi(const Call* calls, int n, const DeviceInfo& dev, int forced, bo
     if (forced != SGMV_VARIANT_SIMT && dev.cc_major == 10) {
         Problem ps[SGMV_MAX_SLICES];
         for (int i = 0; i < n; ++i) ps[i] = calls[i].p;
-        if (tc_supports(ps, n)) {
+        if (tc_supports(ps, n, forced_bn(forced))) {
             *fused = true;
             return SGMV_VARIANT_TC;
         }
@@ -267,15 +271,26 @@ bool bgmv_fast_ok(const Problem& p) {
 int choose_bgmv(const Call& c, int forced) {
     const bool fast = bgmv_fast_ok(c.p);
     if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
-    if (forced == SGMV_VARIANT_TC) return SGMV_ERR_VARIANT;
+    if (forced == SGMV_VARIANT_TC || forced == SGMV_VARIANT_TC_WIDE) return SGMV_ERR_VARIANT;
     if (forced == SGMV_VARIANT_DECODE) return fast ? (int)SGMV_VARIANT_DECODE : (int)SGMV_ERR_VARIANT;
     return fast ? SGMV_VARIANT_DECODE : SGMV_VARIANT_SIMT;
 }
 
+// x can be read as 16-byte pieces of B's dtype straight from its rows.
+bool bgmv_x_vector(const Problem& p) {
+    return p.x_dt == p.w_dt && p.x_cs == 1 && (reinterpret_cast<uintptr_t>(p.x) & 15) == 0 && (p.x_rs * 2) % 16 == 0;
+}
+
 template <int OUT_DT>
 int launch_bgmv_dt(const Problem& p, dim3 grid, cudaStream_t stream) {
-    if (p.add) bgmv_expand_kernel<OUT_DT, true><<<grid, BGMV_THREADS, 0, stream>>>(p);
-    else bgmv_expand_kernel<OUT_DT, false><<<grid, BGMV_THREADS, 0, stream>>>(p);
+    const bool xv = bgmv_x_vector(p);
+    if (p.add) {
+        if (xv) bgmv_expand_kernel<OUT_DT, true, true><<<grid, BGMV_THREADS, 0, stream>>>(p);
+        else bgmv_expand_kernel<OUT_DT, true, false><<<grid, BGMV_THREADS, 0, stream>>>(p);
+    } else {
+        if (xv) bgmv_expand_kernel<OUT_DT, false, true><<<grid, BGMV_THREADS, 0, stream>>>(p);
+        else bgmv_expand_kernel<OUT_DT, false, false><<<grid, BGMV_THREADS, 0, stream>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? SGMV_OK : SGMV_ERR_LAUNCH;
 }
 
@@ -312,7 +327,8 @@ int choose_shrink(const Call& c, const DeviceInfo& dev, int forced, const void* 
     int v;
     if (forced == SGMV_VARIANT_SIMT) v = SGMV_VARIANT_SIMT;
     else if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;
-    else if (forced == SGMV_VARIANT_TC) v = tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
+    else if (forced == SGMV_VARIANT_TC || forced == SGMV_VARIANT_TC_WIDE)
+        v = tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
     else v = tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
     if (v == SGMV_VARIANT_TC && ws) {
         int sp = shr::preferred_splits(c.p, dev.sm_count);
@@ -505,7 +521,7 @@ int sgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lora_b, cons
     const int v = choose_variant(c, dev, forced);
     if (v < 0) return v;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (v == SGMV_VARIANT_TC) return launch_tc(&c.p, 1, dev.sm_count, st);
+    if (v == SGMV_VARIANT_TC) return launch_tc(&c.p, 1, dev.sm_count, st, forced_bn(forced));
     return launch_simt(c, dev, st);
 }
 
@@ -551,11 +567,12 @@ int sgmv_expand_multi_slice(const sgmv_tensor* inputs, const sgmv_tensor* const*
     if (fused) {
         Problem ps[SGMV_MAX_SLICES];
         for (int i = 0; i < n; ++i) ps[i] = calls[i].p;
-        return launch_tc(ps, n, dev.sm_count, st);
+        return launch_tc(ps, n, dev.sm_count, st, forced_bn(forced));
     }
     for (int i = 0; i < n; ++i) {
         const int vi = choose_variant(calls[i], dev, forced);
-        rc = vi == SGMV_VARIANT_TC ? launch_tc(&calls[i].p, 1, dev.sm_count, st) : launch_simt(calls[i], dev, st);
+        rc = vi == SGMV_VARIANT_TC ? launch_tc(&calls[i].p, 1, dev.sm_count, st, forced_bn(forced))
+                                   : launch_simt(calls[i], dev, st);
         if (rc) return rc;
     }
     return SGMV_OK;
@@ -641,7 +658,7 @@ const char* sgmv_status_string(int code) {
 
 int sgmv_set_variant(int variant) {
     if (variant != SGMV_VARIANT_AUTO && variant != SGMV_VARIANT_SIMT && variant != SGMV_VARIANT_TC &&
-        variant != SGMV_VARIANT_DECODE)
+        variant != SGMV_VARIANT_DECODE && variant != SGMV_VARIANT_TC_WIDE)
         return SGMV_ERR_VARIANT;
     return g_forced_variant.exchange(variant);
 }

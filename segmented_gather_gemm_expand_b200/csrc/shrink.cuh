@@ -122,6 +122,12 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
     }
     if (warp == 1) tmem_alloc(smem_u32(&s_tmem_base), (uint32_t)g.tmem_cols);
 
+    // Everything below may read memory written by the preceding kernel.
+    grid_dependency_wait();
+    // The reduction kernel (split H) may be scheduled now; it waits for this
+    // grid to finish before it reads the partial sums.
+    grid_dependents_launch();
+
     // Segment table (guards of sgmv.h applied) and the prefix of row blocks.
     const int32_t nseg = (int32_t)p.batches;
     for (int32_t b = tid; b < nseg; b += THREADS) {
@@ -275,6 +281,7 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
 // into out.  Grid: x = element chunks of a segment, y = segments (grid-stride).
 template <int OUT_DT>
 __global__ void __launch_bounds__(256) shrink_reduce_kernel(Problem p, const float* ws, int splits, int64_t t_lim) {
+    grid_dependency_wait();   // the partial sums of the preceding shrink_kernel grid
     const int64_t R = p.N;
     for (int64_t b = blockIdx.y; b < p.batches; b += gridDim.y) {
         const Segment s = load_segment(p, b);
@@ -298,15 +305,31 @@ struct Plan {
     CUtensorMap am;
 };
 
-// The splits a call would like: enough items (blocks x splits) for two per
-// SM, as a power of two no larger than the chunk count.
+// The splits a call would like (a power of two, at most 16 and at most the
+// chunk count): the one that minimises the bytes the busiest SM moves, i.e.
+// ceil(items / SMs) items of 128 x H/splits x 2 bytes of x, plus its share
+// of the partial sums written and read back (2 x splits x rows x rank x 4
+// bytes over all SMs).  The block count is estimated from the row count and
+// the number of segments (each adds at most one partial block).
 inline int preferred_splits(const Problem& p, int sm_count) {
     const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int64_t blocks = (t_lim + BM - 1) / BM + (p.batches < t_lim ? p.batches : t_lim);
     const int64_t nchunks = (p.K + CH - 1) / CH;
-    int s = 1;
-    while (s < 16 && s * 2 <= nchunks && blocks * s < 2 * (int64_t)sm_count) s *= 2;
-    return s;
+    const int64_t G = sm_count > 0 ? sm_count : 1;
+    int best = 1;
+    double best_cost = 0.0;
+    for (int s = 1; s <= 16 && s <= nchunks; s *= 2) {
+        const int64_t cps = (nchunks + s - 1) / s;
+        const double items_per_sm = (double)((blocks * s + G - 1) / G);
+        const double x_bytes = items_per_sm * BM * (double)cps * CH * 2.0;
+        const double partial = s > 1 ? 2.0 * s * (double)t_lim * (double)p.N * 4.0 / (double)G : 0.0;
+        const double cost = x_bytes + partial;
+        if (s == 1 || cost < best_cost * 0.98) {   // more splits only for a clear gain
+            best = s;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 inline int64_t workspace_bytes_for(const Problem& p, int splits) {
@@ -389,16 +412,34 @@ int launch_dt(const Plan& pl, const Problem& p, float* ws, cudaStream_t stream) 
             return SGMV_ERR_CUDA;
         configured = true;
     }
-    kern<<<pl.grid, THREADS, pl.smem_bytes, stream>>>(pl.xm, pl.am, p, pl.geo, ws);
-    if (cudaGetLastError() != cudaSuccess) return SGMV_ERR_LAUNCH;
+    // Both kernels are launched with programmatic stream serialization: each
+    // may start its prologue while the kernel before it drains, and waits
+    // (griddepcontrol.wait) before it reads global memory.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = (size_t)pl.smem_bytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, pl.xm, pl.am, p, pl.geo, ws) != cudaSuccess) return SGMV_ERR_LAUNCH;
     if (pl.geo.splits > 1) {
         const int64_t rows_guess = (pl.geo.t_lim + p.batches - 1) / (p.batches > 0 ? p.batches : 1);
         int64_t gx = (rows_guess * p.N + 255) / 256;
         if (gx < 1) gx = 1;
         if (gx > 1024) gx = 1024;
-        const dim3 grid((unsigned)gx, (unsigned)(p.batches < 65535 ? p.batches : 65535));
-        shrink_reduce_kernel<OUT_DT><<<grid, 256, 0, stream>>>(p, ws, pl.geo.splits, pl.geo.t_lim);
-        if (cudaGetLastError() != cudaSuccess) return SGMV_ERR_LAUNCH;
+        cudaLaunchConfig_t rc = {};
+        rc.gridDim = dim3((unsigned)gx, (unsigned)(p.batches < 65535 ? p.batches : 65535));
+        rc.blockDim = dim3(256);
+        rc.stream = stream;
+        rc.attrs = attr;
+        rc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&rc, shrink_reduce_kernel<OUT_DT>, p, (const float*)ws, (int)pl.geo.splits,
+                               (int64_t)pl.geo.t_lim) != cudaSuccess)
+            return SGMV_ERR_LAUNCH;
     }
     return SGMV_OK;
 }

@@ -48,7 +48,7 @@ namespace sgmv {
 namespace tc {
 
 constexpr int BM = 128;               // rows per MMA tile (TMEM lanes)
-constexpr int BN = 128;               // columns per n-tile (TMEM columns per accumulator)
+constexpr int TMEM_COLS = 512;       // every accumulator of a CTA: all of TMEM
 constexpr int GROUP = 8;              // rows per work unit
 constexpr int GROUPS_PER_BLOCK = BM / GROUP;
 constexpr int THREADS = 352;
@@ -56,14 +56,13 @@ constexpr int EPI_WARP0 = 3;          // first epilogue warp
 constexpr int EPI_GROUPS = 2;         // epilogue warp groups, taking pieces in turn
 constexpr int EPI_WARPS = 4 * EPI_GROUPS;
 constexpr int SEG_CAP = 1024;         // segments held in shared memory
-constexpr int NUM_ACC = 4;            // TMEM accumulators (4 x 128 columns = all of TMEM)
 constexpr int MAX_KP = 128;           // largest padded rank
 constexpr int NUM_YMAPS = 5;          // output boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
 constexpr int MAX_SLICES = 4;         // slices of one output updated by one launch
 constexpr int RING_PIECES = 32;       // pieces that may hold ring space at once
 // an accumulator slot and a ring barrier slot always serve the same epilogue group
-static_assert(NUM_ACC % EPI_GROUPS == 0 && RING_PIECES % EPI_GROUPS == 0, "slot ownership");
+static_assert(RING_PIECES % EPI_GROUPS == 0, "slot ownership");
 
 struct SegEntry {
     int32_t row0;
@@ -83,6 +82,7 @@ struct Geometry {
     int32_t w_is_bf16;
     int32_t wmin, wfix; // scheduling weight of a piece: max(its 8-row groups, wmin) + wfix
     int32_t rr;         // 1: the kernel may hand out pieces round-robin (see the segment table)
+    int32_t bn;         // columns per n-tile: 128 or 256 (the kernel's BN)
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
     // (rows of 2*kb bytes, swizzled by the row width) at w_blk_off in a stage
     int32_t w_nblk;
@@ -136,7 +136,7 @@ struct Piece {
     int32_t rows;         // rows of the block (1 .. 128)
     int32_t n0;           // first column within the slice
     int32_t col0;         // first output column of the piece
-    int32_t ncols;        // columns of the piece (1 .. BN)
+    int32_t ncols;        // columns of the piece (1 .. the n-tile width)
     int32_t slice;
     int32_t shift;        // TMEM lane of the piece's first row (0, 32, 64 or 96)
     int32_t t;            // index of the piece among this CTA's pieces
@@ -154,6 +154,7 @@ struct Walker {
     const SegEntry* segs;
     const SliceTable* st;   // shared memory
     int32_t nseg, n_tiles, wmin, wfix;
+    int32_t bn;           // columns per n-tile
     int32_t i, rb, j;     // segment, row block, n-tile
     int32_t t;            // pieces handed out so far
     int32_t G, nblk, gcw; // groups and blocks of segment i; weight of a piece of block rb
@@ -270,9 +271,9 @@ struct Walker {
         int32_t sl = 0;
         while (j >= st->tile0[sl + 1]) ++sl;
         p.slice = sl;
-        p.n0 = (j - st->tile0[sl]) * BN;
+        p.n0 = (j - st->tile0[sl]) * bn;
         p.col0 = st->off[sl] + p.n0;
-        p.ncols = min(BN, st->N[sl] - p.n0);
+        p.ncols = min(bn, st->N[sl] - p.n0);
         // Short pieces take turns in the TMEM lane quadrants, so that the
         // epilogue warps of every quadrant share them: the pieces of one
         // epilogue group (every EPI_GROUPS-th) cycle through the quadrants.
@@ -355,12 +356,15 @@ __device__ __forceinline__ int32_t ring_place(int32_t& head, int32_t rows8, int3
 
 // ---------------------------------------------------------------- the kernel
 
-template <int OUT_DT, bool ADD>
+// BN: columns per n-tile (128 or 256); TMEM holds TMEM_COLS / BN accumulators.
+template <int OUT_DT, bool ADD, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ YMaps ymaps, Problem p, Geometry geo,
                        const __grid_constant__ Slices sl) {
     constexpr int OUT_BYTES = OUT_DT == SGMV_F32 ? 4 : 2;
+    constexpr int NUM_ACC = TMEM_COLS / BN;
+    static_assert(NUM_ACC % EPI_GROUPS == 0, "an accumulator slot always serves the same epilogue group");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -433,14 +437,16 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     // chunks past K, and the chunk B's 8-column block points its upper K half at.
     {
         const int kc_real = geo.K / 8, kc_pad = geo.Kp / 8;
-        const int npad = (kc_pad - kc_real) * 128;   // 16-byte rows per buffer (BN == BM == 128)
         for (int b = 0; b < SW + SXO; ++b) {
             uint8_t* buf;
+            int npad;   // 16-byte rows to clear: one per B row (BN) or x row (BM) per missing K chunk
             if (b < SW) {
                 if (geo.w_zero_off < 0) continue;
                 buf = smem + geo.off_w + b * geo.w_bytes + geo.w_zero_off;
+                npad = (kc_pad - kc_real) * BN;
             } else {
-                buf = smem + geo.off_xo + (b - SW) * geo.xo_bytes + kc_real * 128 * 16;
+                buf = smem + geo.off_xo + (b - SW) * geo.xo_bytes + kc_real * BM * 16;
+                npad = (kc_pad - kc_real) * BM;
             }
             for (int q = tid; q < npad; q += THREADS) *reinterpret_cast<uint4*>(buf + q * 16) = make_uint4(0, 0, 0, 0);
         }
@@ -498,6 +504,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     walk.nseg = nseg;
     walk.n_tiles = geo.n_tiles;
     walk.wmin = geo.wmin;
+    walk.bn = BN;
     walk.wfix = geo.wfix;
     if (rr)
         walk.seek_rr((int32_t)blockIdx.x, (int32_t)gridDim.x);
@@ -856,7 +863,8 @@ constexpr int PIECE_FIXED_GROUPS = 0;
 // 128-row pieces, with the deepest B pipeline that leaves it room.
 inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* total_out) {
     const int sw_opts[] = {8, 6, 4, 3, 2};
-    const int32_t row_bytes = BN * out_bytes;              // one ring row across all chunks
+    const int32_t row_bytes = g.bn * out_bytes;            // one ring row across all chunks
+    const int num_acc = TMEM_COLS / g.bn;
     const int32_t budget = SMEM_OPTIN - SMEM_STATIC_RESERVE - 1024;   // 1024: base alignment slack
     for (int prefer_rows : {4 * BM, 3 * BM, 2 * BM, BM}) {
         for (int sw : sw_opts) {
@@ -865,7 +873,7 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* 
             g.stages_xr = g.convert_x ? 1 : 0;
             int32_t fixed = sw * g.w_bytes + g.stages_xo * g.xo_bytes + g.stages_xr * g.xr_bytes +
                             round_up(seg_bytes, 16) + RING_PIECES * 4 +
-                            8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * NUM_ACC + 2 * RING_PIECES) + 64;
+                            8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * num_acc + 2 * RING_PIECES) + 64;
             const int32_t rows = ((budget - fixed) / row_bytes) & ~(GROUP - 1);
             if (rows < prefer_rows) continue;
             g.ring_rows = rows;
@@ -883,7 +891,7 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* 
             g.off_ends = off;
             off += RING_PIECES * 4;
             g.off_bar = round_up(off, 8);
-            off = g.off_bar + 8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * NUM_ACC + 2 * RING_PIECES);
+            off = g.off_bar + 8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * num_acc + 2 * RING_PIECES);
             const int total = off + 1024;
             if (total > SMEM_OPTIN - SMEM_STATIC_RESERVE) continue;
             *total_out = total;
@@ -911,9 +919,9 @@ inline bool slice_ok(const Problem& p) {
 }
 
 // Everything the tensor-core kernel needs for `nsl` slices of one output
-// (sharing x, the metadata and the adapter count), or false if it cannot
-// take the call.
-inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
+// (sharing x, the metadata and the adapter count) with n-tiles of `bn`
+// columns, or false if it cannot take the call.
+inline bool make_plan_bn(const Problem* ps, int nsl, int sm_count, int bn, Plan* out) {
     if (nsl < 1 || nsl > MAX_SLICES) return false;
     const Problem& p = ps[0];
     for (int i = 0; i < nsl; ++i) {
@@ -927,7 +935,7 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     for (int i = 0; i < nsl; ++i) {
         sl.off[i] = ps[i].off;
         sl.N[i] = ps[i].N;
-        sl.tile0[i + 1] = sl.tile0[i] + (int32_t)((ps[i].N + BN - 1) / BN);
+        sl.tile0[i + 1] = sl.tile0[i] + (int32_t)((ps[i].N + bn - 1) / bn);
     }
     for (int i = nsl; i < MAX_SLICES; ++i) {
         sl.off[i] = 0;
@@ -937,8 +945,8 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     const int64_t n_tiles = sl.tile0[nsl];
     const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int64_t max_pieces = (t_lim / BM + p.batches + 1) * n_tiles;
-    const int64_t group_bytes = (int64_t)GROUP * BN * so * (p.add ? 2 : 1);
-    const int64_t wfix = (BN * p.K * 2 + group_bytes - 1) / group_bytes + PIECE_FIXED_GROUPS;
+    const int64_t group_bytes = (int64_t)GROUP * bn * so * (p.add ? 2 : 1);
+    const int64_t wfix = (bn * p.K * 2 + group_bytes - 1) / group_bytes + PIECE_FIXED_GROUPS;
     const int64_t weight_bound = (t_lim / GROUP + p.batches + 1) * n_tiles + (wfix + PIECE_WEIGHT_FLOOR) * max_pieces;
     if (weight_bound >= (int64_t(1) << 31)) return false;
 
@@ -950,6 +958,7 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     g.n_tiles = (int32_t)n_tiles;
     g.w_is_bf16 = p.w_dt == SGMV_BF16;
     g.wmin = PIECE_WEIGHT_FLOOR;
+    g.bn = bn;
     // Round-robin pieces are allowed unless x must be rounded to the weights'
     // dtype: that is done once per x block, so a CTA keeps a block's n-tiles.
     g.rr = g.convert_x ? 0 : 1;
@@ -961,7 +970,7 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
             g.w_blk_k0[nb] = k0;
             g.w_blk_kb[nb] = kb;
             g.w_blk_off[nb] = off;
-            off += round_up(BN * kb * 2, 1024);
+            off += round_up(bn * kb * 2, 1024);
             k0 += kb;
             ++nb;
         };
@@ -973,7 +982,7 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
         g.w_zero_off = -1;
         if (g.w_blk_kb[nb - 1] == 8) {   // the upper K half of the last MMA step reads zeros
             g.w_zero_off = off;
-            off += BN * 16;
+            off += bn * 16;
         }
         g.w_bytes = round_up(off, 1024);
         // B descriptors per K=16 step: swizzle code and 8-row stride follow the
@@ -1012,7 +1021,7 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
         if (p.lora_num == 1) a_stride = (cuuint64_t)round_up((int32_t)(p.N * p.w_ns * 2), 16);
         const cuuint64_t strides[2] = {(cuuint64_t)(p.w_ns * 2), a_stride};
         const int kb = g.w_blk_kb[b];
-        const cuuint32_t box[3] = {(cuuint32_t)kb, (cuuint32_t)BN, 1};
+        const cuuint32_t box[3] = {(cuuint32_t)kb, (cuuint32_t)bn, 1};
         const CUtensorMapSwizzle sw = kb == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                       : kb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                       : kb == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
@@ -1062,9 +1071,37 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out) {
     return true;
 }
 
-template <int OUT_DT, bool ADD>
+// n-tile width of a call.  256-column pieces halve the per-piece work (MMA
+// issue, barriers, TMA requests) and move 512 contiguous bytes of each output
+// row, but a CTA then has half as many pieces, so its pipeline fill and its
+// last piece weigh twice as much; B tiles of 256 rows also crowd the output
+// ring at rank 64 and up.  Measured on one B200 (us per call, 128 vs 256):
+// single-tenant long prefill 66.7 vs 52.0, decode-like mix 80.4 vs 64.7,
+// QKV prefill 30.4 vs 33.9, rank-64 MLP 181 vs 277.  So 256 is taken for
+// ranks up to 32 with x already in B's dtype when the estimated piece count
+// gives every SM at least 16 pieces (overwrite) or 32 (add: loads of the old
+// output also wait in the ring).
+inline int choose_bn(const Problem* ps, int nsl, int sm_count) {
+    const Problem& p = ps[0];
+    if (p.K > 32 || p.x_dt != p.w_dt) return 128;
+    const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
+    int64_t tiles = 0;
+    for (int i = 0; i < nsl; ++i) tiles += (ps[i].N + 255) / 256;
+    const int64_t est = (t_lim / BM + p.batches) * tiles;
+    return est >= (p.add ? 32 : 16) * (int64_t)sm_count ? 256 : 128;
+}
+
+// force_bn: 0 lets choose_bn decide; 128 or 256 fixes the width.
+inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out, int force_bn = 0) {
+    if (nsl < 1 || nsl > MAX_SLICES) return false;
+    if (force_bn) return make_plan_bn(ps, nsl, sm_count, force_bn, out);
+    if (choose_bn(ps, nsl, sm_count) == 256 && make_plan_bn(ps, nsl, sm_count, 256, out)) return true;
+    return make_plan_bn(ps, nsl, sm_count, 128, out);
+}
+
+template <int OUT_DT, bool ADD, int BN>
 int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
-    auto kern = tc_expand_slice_kernel<OUT_DT, ADD>;
+    auto kern = tc_expand_slice_kernel<OUT_DT, ADD, BN>;
     static std::atomic<bool> configured{false};
     if (!configured.load()) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1088,26 +1125,31 @@ int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
 
 }  // namespace tc
 
-bool tc_supports(const Problem* ps, int nsl) {
+bool tc_supports(const Problem* ps, int nsl, int force_bn) {
     tc::Plan pl;
-    return tc::make_plan(ps, nsl, 148, &pl);
+    return tc::make_plan(ps, nsl, 148, &pl, force_bn);
 }
 
-int launch_tc(const Problem* ps, int nsl, int sm_count, cudaStream_t stream) {
-    tc::Plan pl;
-    if (!tc::make_plan(ps, nsl, sm_count, &pl)) return SGMV_ERR_VARIANT;
-    const Problem& p = ps[0];
+template <int BN>
+int launch_bn(const tc::Plan& pl, const Problem& p, cudaStream_t stream) {
     switch (p.out_dt) {
         case SGMV_F32:
-            return p.add ? tc::launch_instance<SGMV_F32, true>(pl, p, stream)
-                         : tc::launch_instance<SGMV_F32, false>(pl, p, stream);
+            return p.add ? tc::launch_instance<SGMV_F32, true, BN>(pl, p, stream)
+                         : tc::launch_instance<SGMV_F32, false, BN>(pl, p, stream);
         case SGMV_BF16:
-            return p.add ? tc::launch_instance<SGMV_BF16, true>(pl, p, stream)
-                         : tc::launch_instance<SGMV_BF16, false>(pl, p, stream);
+            return p.add ? tc::launch_instance<SGMV_BF16, true, BN>(pl, p, stream)
+                         : tc::launch_instance<SGMV_BF16, false, BN>(pl, p, stream);
         default:
-            return p.add ? tc::launch_instance<SGMV_F16, true>(pl, p, stream)
-                         : tc::launch_instance<SGMV_F16, false>(pl, p, stream);
+            return p.add ? tc::launch_instance<SGMV_F16, true, BN>(pl, p, stream)
+                         : tc::launch_instance<SGMV_F16, false, BN>(pl, p, stream);
     }
+}
+
+int launch_tc(const Problem* ps, int nsl, int sm_count, cudaStream_t stream, int force_bn) {
+    tc::Plan pl;
+    if (!tc::make_plan(ps, nsl, sm_count, &pl, force_bn)) return SGMV_ERR_VARIANT;
+    const Problem& p = ps[0];
+    return pl.geo.bn == 256 ? launch_bn<256>(pl, p, stream) : launch_bn<128>(pl, p, stream);
 }
 
 }  // namespace sgmv

@@ -15,7 +15,7 @@ from sgmv_testlib import DeviceProblem, compare, from_torch, to_torch, written_r
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = {"simt": sg.VARIANT_SIMT, "tc": sg.VARIANT_TC}
+VARIANTS = {"simt": sg.VARIANT_SIMT, "tc": sg.VARIANT_TC, "tc_wide": sg.VARIANT_TC_WIDE}
 
 
 @pytest.fixture(autouse=True)
@@ -335,3 +335,23 @@ def test_validate_metadata_bits():
     st = run([10, 0], [4, 6], [0, 1])
     assert st & 16 and not st & 8
     assert run([4, 0], [6, 6], [0, 1]) & 8
+
+
+@pytest.mark.parametrize("case", ["multi_tile_ragged", "wide_slice", "odd_offset_f32_out", "overwrite_mode"])
+def test_tile_widths_give_identical_bits(case):
+    """128- and 256-column n-tiles run the same MMA steps for every output element, so the results
+    must agree bit for bit (this is what lets the library pick the width per call)."""
+    p = gen.custom(seed=sum(map(ord, case)) % 1000, **EDGE[case])
+    outs = []
+    for v in (sg.VARIANT_TC, sg.VARIANT_TC_WIDE):
+        dp = DeviceProblem(p)
+        sg.set_variant(v)
+        try:
+            dp.plan(0)
+        except sg.SgmvError as e:
+            pytest.skip(f"variant {v} does not take this case ({e.code})")
+        dp.run(0)
+        torch.cuda.synchronize()
+        outs.append(dp.result())
+    assert sg.device_error() == 0
+    assert np.array_equal(outs[0], outs[1])

@@ -77,8 +77,10 @@ def test_two_calls_in_a_row_match_the_workspace_entry_point(case):
 
 def test_a_call_needing_more_scratch_is_refused():
     sg.set_variant(sg.VARIANT_AUTO)
-    p = shrink_problem(33, [20000], H=128, R=128, A=1, out_dt="f32")   # 2 splits x 20000 rows x 128 x 4 B > 8 MiB
+    p = shrink_problem(33, [2100], H=4096, R=128, A=1, out_dt="f32")   # splits x 2100 rows x 128 x 4 B > 8 MiB
     x, a, y, meta = device_args(p)
+    _, splits, pref = sg.shrink_plan(x, a, y, *meta, p.batches, p.max_seq_len, 1 << 40)
+    assert pref > _abi_static_bytes(), (splits, pref)
     rc = static_scratch_call(x, a, y, meta, p)
     assert rc == _abi.STATUS["SGMV_ERR_SCRATCH"]
     torch.cuda.synchronize()

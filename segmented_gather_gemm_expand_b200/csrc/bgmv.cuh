@@ -15,7 +15,9 @@
 // are summed in fp32 in k order and the result (plus the old value in add
 // mode) is rounded once.
 //
-// Grid: x = 256-column tile of the slice, y = rows (grid-stride).
+// Grid: x = 256-column tile of the slice, y = rows (grid-stride).  The kernel
+// is launched as a programmatic dependent launch and waits for the preceding
+// kernel's memory before its first global read.
 #pragma once
 
 #include "common.cuh"
@@ -48,6 +50,7 @@ bgmv_expand_kernel(Problem p) {
     const bool mine = n < p.N;
     const bool two = n + 1 < p.N;
 
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // launched as a programmatic dependent launch
     for (int64_t b = blockIdx.y; b < p.batches; b += gridDim.y) {
         const int64_t a = load_meta(p.idx, b);
         if (a < 0 || a >= p.lora_num || b >= lim) continue;     // uniform across the CTA
@@ -98,3 +101,4 @@ bgmv_expand_kernel(Problem p) {
 }
 
 }  // namespace sgmv
+

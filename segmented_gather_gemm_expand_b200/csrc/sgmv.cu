@@ -281,17 +281,30 @@ bool bgmv_x_vector(const Problem& p) {
     return p.x_dt == p.w_dt && p.x_cs == 1 && (reinterpret_cast<uintptr_t>(p.x) & 15) == 0 && (p.x_rs * 2) % 16 == 0;
 }
 
+// Launched as a programmatic dependent launch: the kernel waits for the
+// preceding kernel's memory (griddepcontrol.wait) before its first read.
+template <int OUT_DT, bool ADD, bool XVEC>
+int launch_bgmv_kernel(const Problem& p, dim3 grid, cudaStream_t stream) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(BGMV_THREADS);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, bgmv_expand_kernel<OUT_DT, ADD, XVEC>, p) == cudaSuccess ? SGMV_OK
+                                                                                            : SGMV_ERR_LAUNCH;
+}
+
 template <int OUT_DT>
 int launch_bgmv_dt(const Problem& p, dim3 grid, cudaStream_t stream) {
     const bool xv = bgmv_x_vector(p);
-    if (p.add) {
-        if (xv) bgmv_expand_kernel<OUT_DT, true, true><<<grid, BGMV_THREADS, 0, stream>>>(p);
-        else bgmv_expand_kernel<OUT_DT, true, false><<<grid, BGMV_THREADS, 0, stream>>>(p);
-    } else {
-        if (xv) bgmv_expand_kernel<OUT_DT, false, true><<<grid, BGMV_THREADS, 0, stream>>>(p);
-        else bgmv_expand_kernel<OUT_DT, false, false><<<grid, BGMV_THREADS, 0, stream>>>(p);
-    }
-    return cudaGetLastError() == cudaSuccess ? SGMV_OK : SGMV_ERR_LAUNCH;
+    if (p.add) return xv ? launch_bgmv_kernel<OUT_DT, true, true>(p, grid, stream)
+                         : launch_bgmv_kernel<OUT_DT, true, false>(p, grid, stream);
+    return xv ? launch_bgmv_kernel<OUT_DT, false, true>(p, grid, stream)
+              : launch_bgmv_kernel<OUT_DT, false, false>(p, grid, stream);
 }
 
 int launch_bgmv(const Call& c, cudaStream_t stream) {

@@ -402,27 +402,19 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             s_sl.off[i] = (int32_t)sl.off[i];
             s_sl.N[i] = (int32_t)sl.N[i];
         }
-        for (int i = 0; i < SW; ++i) {
-            mbar_init(smem_u32(&w_full[i]), 1);
-            mbar_init(smem_u32(&w_empty[i]), 1);
+    }
+    {
+        // The barriers lie back to back from w_full; every thread initialises a
+        // few.  acc_empty and y_free count the four warps of an epilogue group.
+        const int n_bars = (int)(y_free + RING_PIECES - bars);
+        const int acc_empty0 = (int)(acc_empty - bars), y_free0 = (int)(y_free - bars);
+        bool did = false;
+        for (int b = tid; b < n_bars; b += THREADS) {
+            const bool four = (b >= acc_empty0 && b < acc_empty0 + NUM_ACC) || b >= y_free0;
+            mbar_init(smem_u32(&bars[b]), four ? 4u : 1u);
+            did = true;
         }
-        for (int i = 0; i < SXO; ++i) {
-            mbar_init(smem_u32(&xo_full[i]), 1);
-            mbar_init(smem_u32(&xo_empty[i]), 1);
-        }
-        for (int i = 0; i < SXR; ++i) {
-            mbar_init(smem_u32(&xr_full[i]), 1);
-            mbar_init(smem_u32(&xr_empty[i]), 1);
-        }
-        for (int i = 0; i < NUM_ACC; ++i) {
-            mbar_init(smem_u32(&acc_full[i]), 1);
-            mbar_init(smem_u32(&acc_empty[i]), 4);      // the four warps of one epilogue group
-        }
-        for (int i = 0; i < RING_PIECES; ++i) {
-            mbar_init(smem_u32(&y_full[i]), 1);
-            mbar_init(smem_u32(&y_free[i]), 4);
-        }
-        fence_barrier_init();
+        if (did) fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_x);
@@ -449,6 +441,15 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 npad = (kc_pad - kc_real) * BM;
             }
             for (int q = tid; q < npad; q += THREADS) *reinterpret_cast<uint4*>(buf + q * 16) = make_uint4(0, 0, 0, 0);
+        }
+    }
+
+    // Warm L2 with the metadata while the preceding kernel may still run.
+    for (int32_t b = tid; b < (int32_t)p.batches; b += THREADS) {
+        for (const MetaVec* m : {&p.start, &p.len, &p.idx}) {
+            if (m->dtype != SGMV_I32 && m->dtype != SGMV_I64) continue;
+            const int64_t esz = m->dtype == SGMV_I64 ? 8 : 4;
+            prefetch_l2(static_cast<const char*>(m->ptr) + b * m->stride * esz);
         }
     }
 

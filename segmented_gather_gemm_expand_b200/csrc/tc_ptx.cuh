@@ -257,6 +257,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int3
         : "memory");
 }
 
+// Hint that a global line will be read soon: fetch it into L2.  Safe on data
+// the preceding kernel may still write (L2 is where writes land; nothing is
+// returned to the thread).
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(ptr)) : "memory");
+}
+
 // Programmatic dependent launch: wait until the preceding grid's memory is
 // visible / allow the next grid to start its prologue.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

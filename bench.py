@@ -316,13 +316,28 @@ def bench_ours(args, rank, world, device):
     variant_name = {1: "simt", 2: "tc", 3: "decode"}.get(v_used, str(v_used))
     # kernel launches one call makes (a split shrink adds the partial-sum reduction)
     launches_per_call = 2 if (p.op == "shrink" and shrink_splits > 1) else 1
+    # One step: the slice calls one by one, or (--step fused) all slices in one
+    # sgmv_expand_multi_slice call.
+    fused_step = args.step == "fused" and ncalls > 1 and p.op == "slice"
+    if fused_step:
+        run_multi_step = make_multi_call(p, (x, ws, y, meta))
+        _, launches_per_step = sg.plan_multi_slice(x, ws, y, *meta, p.batches, p.max_seq_len,
+                                                   [c.slice_offset for c in p.calls], p.add_inputs)
+
+        def step_fn(st):
+            run_multi_step(st)
+    else:
+        launches_per_step = ncalls * launches_per_call
+
+        def step_fn(st):
+            for c in range(ncalls):
+                run(c, st)
 
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            for c in range(ncalls):
-                run(c, stream.cuda_stream)
+            step_fn(stream.cuda_stream)
     torch.cuda.synchronize()
 
     # Capture the timed steps as graphs of back-to-back launches.
@@ -335,8 +350,7 @@ def bench_ours(args, rank, world, device):
         with torch.cuda.graph(g, stream=stream):
             cs = torch.cuda.current_stream().cuda_stream
             for _ in range(s):
-                for c in range(ncalls):
-                    run(c, cs)
+                step_fn(cs)
         graphs.append(g)
         remaining -= s
     # one untimed replay of every graph (first-launch costs)
@@ -374,12 +388,13 @@ def bench_ours(args, rank, world, device):
     assert sg.device_error(device) == 0, "a kernel reported a device-side error"
 
     step_bytes, step_flops, step_rows = step_accounting(p)
-    call_bytes, _, _ = call_accounting(p, 0)
+    calls_per_step = 1 if fused_step else ncalls
+    call_bytes = step_bytes if fused_step else call_accounting(p, 0)[0]
     total_ms, all_bytes, all_flops, all_tokens = reduce_over_ranks(total_ms, step_bytes, step_flops,
                                                                    p.total_tokens, device, world)
     ms_per_step = total_ms / K
     value = all_bytes * K / (total_ms * 1e-3) / 1e9
-    avg_launch_ms = total_ms / (K * ncalls)
+    avg_launch_ms = total_ms / (K * calls_per_step)
     achieved = call_bytes / (avg_launch_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
 
@@ -407,8 +422,7 @@ def bench_ours(args, rank, world, device):
                     w.copy_(pw, non_blocking=True)
                 for m, pm in zip(meta, phmeta):
                     m.copy_(pm, non_blocking=True)
-                for c in range(ncalls):
-                    run(c, stream.cuda_stream)
+                step_fn(stream.cuda_stream)
                 out_host.copy_(y, non_blocking=True)
             e1.record(stream)
         torch.cuda.synchronize()
@@ -420,7 +434,7 @@ def bench_ours(args, rank, world, device):
 
     # ---- the same step as ONE fused multi-slice launch (several slices only)
     fused = None
-    if ncalls > 1 and not args.no_fused:
+    if ncalls > 1 and not args.no_fused and not fused_step:
         run_multi = make_multi_call(p, (x, ws, y, meta))
         fv, fl = sg.plan_multi_slice(x, ws, y, *meta, p.batches, p.max_seq_len,
                                      [c.slice_offset for c in p.calls], p.add_inputs)
@@ -458,9 +472,11 @@ def bench_ours(args, rank, world, device):
                    "parallelism": f"replicas x{world} (independent batches, no collective)",
                    "l2": "no flush: every step streams the whole output, larger than L2",
                    "variant": variant_name, "seed": args.seed,
+                   "step": ("all slices in one sgmv_expand_multi_slice call" if fused_step else
+                            f"{ncalls} separate call(s)"),
                    "timing": f"CUDA graphs of <= {STEPS_PER_GRAPH} steps; events around the timed region"},
-        "tokens_per_s": all_tokens * ncalls / (total_ms * 1e-3) / ncalls,
-        "tokens_per_s_note": "tokens of one call / average call time (per call, all ranks)",
+        "tokens_per_s": all_tokens * K / (total_ms * 1e-3),
+        "tokens_per_s_note": "batch tokens per second, all ranks (a step updates every slice of every token)",
         "tflops": all_flops * K / (total_ms * 1e-3) / 1e12,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(args.workload, variant_name),
@@ -469,10 +485,10 @@ def bench_ours(args, rank, world, device):
                      "kernel": f"{ {'bgmv': 'bgmv_expand_slice', 'shrink': 'sgmv_shrink'}.get(p.op, 'sgmv_expand_slice') } "
                                f"({variant_name}{', %d H splits + reduction' % shrink_splits if shrink_splits > 1 else ''})",
                      "launch_ms_avg": avg_launch_ms, "bytes_per_launch": call_bytes,
-                     "launches_timed": K * ncalls,
+                     "launches_timed": K * calls_per_step,
                      "launch_ms_note": "timed region / calls (back-to-back calls, gaps included; a split shrink "
                                        "call is its main kernel plus the reduction)"},
-        "gpu_launches": K * ncalls * launches_per_call,
+        "gpu_launches": K * launches_per_step,
         "clocks": clocks,
         "fused_multi_slice": fused,
         "e2e": e2e,
@@ -585,6 +601,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the extra timing of the step as one multi-slice call")
+    ap.add_argument("--step", choices=["calls", "fused"], default="calls",
+                    help="time each step as separate slice calls (default) or as one multi-slice call")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

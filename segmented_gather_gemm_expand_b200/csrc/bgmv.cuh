@@ -100,5 +100,76 @@ bgmv_expand_kernel(Problem p) {
     }
 }
 
-}  // namespace sgmv
+// ----------------------------------------------------------------------------
+// Coalesced variant for ranks that are powers of two (8 .. 256).  A warp load
+// of the kernel above touches 32 different 128-byte lines (thread t reads its
+// own two B rows), so the L1 tag stage, not DRAM, sets its pace.  Here a warp
+// covers 64 B rows of the CTA's 256 and every one of its 16-byte loads reads
+// 512 contiguous bytes: K/8 threads share a row, each taking one 16-byte chunk
+// (eight ranks), and the row's sum is completed with shuffles.  The 256 sums
+// go through shared memory to coalesced output stores.  (Two token rows per CTA
+// step, with both rows' loads in flight, measured slower: the register cost
+// halves the CTAs an SM holds.)
+template <int OUT_DT, bool ADD>
+__global__ void __launch_bounds__(BGMV_THREADS)
+bgmv_coalesced_kernel(Problem p) {
+    __shared__ float res[BGMV_COLS];
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const bool w_bf16 = p.w_dt == SGMV_BF16;
+    const int K = (int)p.K;
+    const int tpr = K / 8;                      // threads per B row (1 .. 32)
+    const int rpi = 32 / tpr;                   // rows per warp load
+    const int chunk = lane % tpr;               // this thread's 16-byte chunk of a row
+    const int64_t n0 = (int64_t)blockIdx.x * BGMV_COLS;
+    const int64_t lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
+    const uint16_t* wbase = static_cast<const uint16_t*>(p.w);
+    const int loads = 64 / rpi;                 // warp loads covering the warp's 64 rows
 
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // launched as a programmatic dependent launch
+    for (int64_t b = blockIdx.y; b < p.batches; b += gridDim.y) {
+        const int64_t a = load_meta(p.idx, b);
+        if (a < 0 || a >= p.lora_num || b >= lim) continue;     // uniform across the CTA
+        // this thread's eight ranks of x, rounded to B's dtype
+        float xv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xv[e] = round_to(load_elem(p.x, p.x_dt, b * p.x_rs + (chunk * 8 + e) * p.x_cs), p.w_dt);
+        const uint16_t* wa = wbase + a * p.w_as;
+        for (int l0 = 0; l0 < loads; l0 += 8) {
+            uint4 v[8];
+            float part[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t r = n0 + warp * 64 + (int64_t)(l0 + u) * rpi + lane / tpr;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (l0 + u < loads && r < p.N)
+                    v[u] = __ldg(reinterpret_cast<const uint4*>(wa + r * p.w_ns) + chunk);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc = fmaf(xv[e], half8_elem(v[u], e, w_bf16), acc);
+                part[u] = acc;
+            }
+            for (int o = tpr / 2; o >= 1; o /= 2) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
+            }
+            if (chunk == 0) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (l0 + u < loads) res[warp * 64 + (l0 + u) * rpi + lane / tpr] = part[u];
+            }
+        }
+        __syncthreads();
+        const int64_t oi = b * p.H + p.off + n0;
+        for (int c = tid; c < BGMV_COLS; c += BGMV_THREADS) {
+            if (n0 + c >= p.N) break;
+            const float v = res[c];
+            store_elem(p.out, OUT_DT, oi + c, ADD ? load_elem(p.out, OUT_DT, oi + c) + v : v);
+        }
+        __syncthreads();   // res is read before the next row overwrites it
+    }
+}
+
+}  // namespace sgmv

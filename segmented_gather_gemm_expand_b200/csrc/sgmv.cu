@@ -307,8 +307,34 @@ int launch_bgmv_dt(const Problem& p, dim3 grid, cudaStream_t stream) {
               : launch_bgmv_kernel<OUT_DT, false, false>(p, grid, stream);
 }
 
+// Ranks that are powers of two take the coalesced kernel (every warp load reads
+// 512 contiguous bytes of B); the others the two-rows-per-thread kernel.
+template <int OUT_DT>
+int launch_bgmv_coalesced(const Problem& p, dim3 grid, cudaStream_t stream) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(BGMV_THREADS);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = p.add ? cudaLaunchKernelEx(&cfg, bgmv_coalesced_kernel<OUT_DT, true>, p)
+                                : cudaLaunchKernelEx(&cfg, bgmv_coalesced_kernel<OUT_DT, false>, p);
+    return e == cudaSuccess ? SGMV_OK : SGMV_ERR_LAUNCH;
+}
+
 int launch_bgmv(const Call& c, cudaStream_t stream) {
     const Problem& p = c.p;
+    if ((p.K & (p.K - 1)) == 0) {
+        dim3 grid((unsigned)((p.N + BGMV_COLS - 1) / BGMV_COLS), (unsigned)(p.batches < 65535 ? p.batches : 65535));
+        switch (p.out_dt) {
+            case SGMV_F32: return launch_bgmv_coalesced<SGMV_F32>(p, grid, stream);
+            case SGMV_BF16: return launch_bgmv_coalesced<SGMV_BF16>(p, grid, stream);
+            default: return launch_bgmv_coalesced<SGMV_F16>(p, grid, stream);
+        }
+    }
     dim3 grid((unsigned)((p.N + BGMV_COLS - 1) / BGMV_COLS), (unsigned)(p.batches < 65535 ? p.batches : 65535));
     switch (p.out_dt) {
         case SGMV_F32: return launch_bgmv_dt<SGMV_F32>(p, grid, stream);

@@ -18,7 +18,10 @@
 //                        into one of four TMEM accumulators.
 //   warps 3-10 epilogue  two groups of four warps take alternate pieces; warp w
 //                        owns TMEM lanes 32*(w%4).. (32 rows of the piece) and
-//                        all its columns: tcgen05.ld the fp32 sums, add
+//                        all its columns, or, for a piece of at most 64 rows
+//                        (computed once per 32- or 64-lane span), its rows in
+//                        its span and every 2nd or 4th column chunk: tcgen05.ld
+//                        the fp32 sums, add
 //                        the old output (add mode), round once to the output
 //                        dtype, write the tile back in place in shared memory
 //                        and TMA-store its whole 8-row groups; the last < 8
@@ -48,6 +51,8 @@ namespace sgmv {
 namespace tc {
 
 constexpr int BM = 128;               // rows per MMA tile (TMEM lanes)
+constexpr int BM_LOG = 7;
+static_assert((1 << BM_LOG) == BM, "BM is a power of two");
 constexpr int TMEM_COLS = 512;       // every accumulator of a CTA: all of TMEM
 constexpr int GROUP = 8;              // rows per work unit
 constexpr int GROUPS_PER_BLOCK = BM / GROUP;
@@ -138,11 +143,17 @@ struct Piece {
     int32_t col0;         // first output column of the piece
     int32_t ncols;        // columns of the piece (1 .. the n-tile width)
     int32_t slice;
-    int32_t shift;        // TMEM lane of the piece's first row (0, 32, 64 or 96)
+    int32_t rep_log;      // log2 of the copies of the piece's rows in TMEM (1, 2 or 4 copies,
+                          // one per 128/copies lanes)
+    int32_t shift;        // lane of the piece's first row within each copy (0, 32, 64 or 96)
     int32_t t;            // index of the piece among this CTA's pieces
     bool new_x;           // first piece of this x block in this CTA
     bool last_x;          // last piece of this x block in this CTA
 };
+
+// log2 of the lanes between repeats of a block's rows in the staged x operand:
+// the rows rounded up to 32, 64 or 128.
+__device__ __forceinline__ int32_t x_period_log(int32_t rows) { return rows <= 32 ? 5 : rows <= 64 ? 6 : BM_LOG; }
 
 // Walks the CTA's pieces in one of two ways:
 //   - contiguous: the pieces whose start weight lies in [w0, w_end) (seek);
@@ -155,6 +166,7 @@ struct Walker {
     const SliceTable* st;   // shared memory
     int32_t nseg, n_tiles, wmin, wfix;
     int32_t bn;           // columns per n-tile
+    int32_t cc_log;       // log2 of the columns per 128-byte output chunk
     int32_t i, rb, j;     // segment, row block, n-tile
     int32_t t;            // pieces handed out so far
     int32_t G, nblk, gcw; // groups and blocks of segment i; weight of a piece of block rb
@@ -274,12 +286,20 @@ struct Walker {
         p.n0 = (j - st->tile0[sl]) * bn;
         p.col0 = st->off[sl] + p.n0;
         p.ncols = min(bn, st->N[sl] - p.n0);
-        // Short pieces take turns in the TMEM lane quadrants, so that the
-        // epilogue warps of every quadrant share them: the pieces of one
-        // epilogue group (every EPI_GROUPS-th) cycle through the quadrants.
-        const int32_t nq = (p.rows + 31) / 32;
-        const int32_t turn = t / EPI_GROUPS;
-        p.shift = nq == 1 ? 32 * (turn % 4) : nq == 2 ? 64 * (turn % 2) : 0;
+        // A short piece (rows in 1 or 2 quadrants) is computed in every span
+        // of 32 or 64 lanes: the x block is staged with its rows repeated
+        // (x_period), so each TMEM quadrant holds a copy of the sums, and the
+        // epilogue warps of the copies split the piece's column chunks.  Where
+        // the piece has fewer chunks than copies, its rows instead take turns
+        // in the lanes of a wider span (the pieces of one epilogue group,
+        // every EPI_GROUPS-th, cycle through them).
+        // (all powers of two: shifts and masks only, this runs for every piece in every role)
+        const int32_t span_log = x_period_log(p.rows);
+        const int32_t nch = (p.ncols + (1 << cc_log) - 1) >> cc_log;
+        const int32_t maxrep_log = BM_LOG - span_log;
+        p.rep_log = min(maxrep_log, nch >= 4 ? 2 : nch >= 2 ? 1 : 0);
+        const int32_t turns_mask = (1 << (maxrep_log - p.rep_log)) - 1;
+        p.shift = ((t / EPI_GROUPS) & turns_mask) << span_log;
         p.t = t++;
     }
 
@@ -506,6 +526,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     walk.n_tiles = geo.n_tiles;
     walk.wmin = geo.wmin;
     walk.bn = BN;
+    walk.cc_log = OUT_BYTES == 4 ? 5 : 6;
     walk.wfix = geo.wfix;
     if (rr)
         walk.seek_rr((int32_t)blockIdx.x, (int32_t)gridDim.x);
@@ -620,12 +641,14 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             if (pc.new_x) {
                 xcur = xb++;
                 const int xs = xcur % SXO;
+                const int pmask = (1 << x_period_log(pc.rows)) - 1;   // operand row m holds x row m % period
                 if (geo.convert_x) {
                     const int rs = xcur % SXR;
                     if (!warp_wait(smem_u32(&xr_full[rs]), (xcur / SXR) & 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
                     if (!warp_wait(smem_u32(&xo_empty[xs]), ((xcur / SXO) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_MMA))
                         break;
-                    // x (its own dtype, row-major) -> weights' dtype, K-major core matrices
+                    // x (its own dtype, row-major) -> weights' dtype, K-major core matrices,
+                    // the block's rows repeated every period
                     const uint8_t* xraw = smem + geo.off_xr + rs * geo.xr_bytes;
                     uint8_t* xop = smem + geo.off_xo + xs * geo.xo_bytes;
                     const int row_bytes = geo.K * geo.x_bytes;
@@ -634,7 +657,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                         uint4 outv = make_uint4(0, 0, 0, 0);
                         if (kc < kc_real) {
                             float f[8];
-                            const uint8_t* src = xraw + m * row_bytes + kc * 8 * geo.x_bytes;
+                            const uint8_t* src = xraw + (m & pmask) * row_bytes + kc * 8 * geo.x_bytes;
                             if (geo.x_bytes == 4) {
                                 const float4 a = *reinterpret_cast<const float4*>(src);
                                 const float4 b = *reinterpret_cast<const float4*>(src + 16);
@@ -661,6 +684,19 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     if (lane == 0) mbar_arrive(smem_u32(&xr_empty[rs]));
                 } else {
                     if (!warp_wait(smem_u32(&xo_full[xs]), (xcur / SXO) & 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
+                    if (pmask < BM - 1) {
+                        // repeat the block's first rows over the whole operand (16-byte
+                        // row pieces; K-block kc of row m at kc * BM * 16 + m * 16)
+                        uint8_t* xop = smem + geo.off_xo + xs * geo.xo_bytes;
+                        const int per = pmask + 1, copies = BM - per;
+                        for (int q = lane; q < copies * kc_pad; q += 32) {
+                            const int kc = q / copies, m = per + q % copies;
+                            *reinterpret_cast<uint4*>(xop + kc * (BM * 16) + m * 16) =
+                                *reinterpret_cast<const uint4*>(xop + kc * (BM * 16) + (m & pmask) * 16);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
                 }
             }
             const int xs = xcur % SXO;
@@ -670,10 +706,9 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             if (!warp_wait(smem_u32(&acc_empty[as]), ((t / NUM_ACC) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
             tc_fence_after();
             if (lane == 0) {
-                // A row m reads x row m - shift: the piece's rows land in TMEM lanes
-                // [shift, shift + rows); rows below come from unrelated shared memory
-                // and only fill lanes nobody reads.
-                const uint32_t a_base = smem_u32(smem + geo.off_xo + xs * geo.xo_bytes) - (uint32_t)(pc.shift * 16);
+                // A row m holds x row m % period: every span of `period` TMEM lanes
+                // receives the piece's sums (lanes past its rows are never read)
+                const uint32_t a_base = smem_u32(smem + geo.off_xo + xs * geo.xo_bytes);
                 const uint32_t b_base = smem_u32(smem + geo.off_w + ws * geo.w_bytes);
                 const uint32_t d = tmem_base + (uint32_t)(as * BN);
 #pragma unroll
@@ -716,14 +751,19 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             const int full_end = pc.rows & ~(GROUP - 1);
             const int ncols = pc.ncols;
             const int64_t col0 = pc.col0;   // first output column of the piece
-            const int pr = r - pc.shift;        // this thread's row within the piece
+            // this warp's copy of the piece (lanes [k * span, (k + 1) * span)) and
+            // its column chunks k, k + rep, ...
+            const int span_log = BM_LOG - pc.rep_log;
+            const int k_copy = (q * 32) >> span_log;
+            const int lane0 = ((q * 32) & ((1 << span_log) - 1)) - pc.shift;   // row of this warp's lane 0 within the piece
+            const int pr = lane0 + lane;        // this thread's row within the piece
             const bool valid = pr >= 0 && pr < pc.rows;
             // rows past the last whole group go straight to global memory from registers
             const bool tail = pr >= full_end;
             uint8_t* ring = smem + geo.off_y;
             const uint32_t taddr = tmem_base + (uint32_t)(as * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-            for (int c = 0; c < NCH; ++c) {
+            for (int c = k_copy; c < NCH; c += 1 << pc.rep_log) {
                 if (c * CC >= ncols) break;     // warp-uniform
                 uint32_t v[CC];
 #pragma unroll
@@ -788,8 +828,8 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             __syncwarp();
             if (lane == 0) {
                 const int32_t xcol0 = (int32_t)col0;
-                const int q_lo = max(q * 32 - pc.shift, 0), q_full = min(q * 32 + 32 - pc.shift, full_end);
-                for (int c = 0; c < NCH; ++c) {
+                const int q_lo = max(lane0, 0), q_full = min(lane0 + 32, full_end);
+                for (int c = k_copy; c < NCH; c += 1 << pc.rep_log) {
                     if (c * CC >= ncols) break;
                     for (int rr = q_lo; rr < q_full;) {
                         const int k = box_level(q_full - rr, 2);

@@ -901,14 +901,23 @@ constexpr int PIECE_WEIGHT_FLOOR = 16;
 constexpr int PIECE_FIXED_GROUPS = 0;
 
 // Shared-memory layout: an output ring of at least 4, else 3, 2, 1 whole
-// 128-row pieces, with the deepest B pipeline that leaves it room.
-inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, int* total_out) {
-    const int sw_opts[] = {8, 6, 4, 3, 2};
+// 128-row pieces, with the deepest B pipeline that leaves it room.  In add
+// mode the ring also holds the old output loaded ahead of the epilogue, and the
+// loads it can keep in flight set the pace: two B stages, the rest for the
+// ring (measured on one B200, us per call, 2 B stages against the deepest
+// that fits: rank-64 MLP 169.4 vs 178.3; QKV prefill and the decode-like mix
+// unchanged; overwrite mode is better with the deep B pipeline).
+inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, bool add, int* total_out) {
+    const int sw_deep[] = {8, 6, 4, 3, 2};
+    const int sw_two[] = {2};
+    const int* sw_opts = add ? sw_two : sw_deep;
+    const int n_sw = add ? 1 : 5;
     const int32_t row_bytes = g.bn * out_bytes;            // one ring row across all chunks
     const int num_acc = TMEM_COLS / g.bn;
     const int32_t budget = SMEM_OPTIN - SMEM_STATIC_RESERVE - 1024;   // 1024: base alignment slack
     for (int prefer_rows : {4 * BM, 3 * BM, 2 * BM, BM}) {
-        for (int sw : sw_opts) {
+        for (int si = 0; si < n_sw; ++si) {
+            const int sw = sw_opts[si];
             g.stages_w = sw;
             g.stages_xo = 2;
             g.stages_xr = g.convert_x ? 1 : 0;
@@ -1048,7 +1057,7 @@ inline bool make_plan_bn(const Problem* ps, int nsl, int sm_count, int bn, Plan*
     g.xo_bytes = BM * g.Kp * 2;
     g.xr_bytes = round_up(BM * (int32_t)p.K * (int32_t)sx, 1024);
     const int32_t seg_bytes = round_up((int32_t)p.batches * (int32_t)sizeof(SegEntry), 16);
-    if (!layout_smem(g, seg_bytes, (int32_t)so, &out->smem_bytes)) return false;
+    if (!layout_smem(g, seg_bytes, (int32_t)so, p.add, &out->smem_bytes)) return false;
 
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;

@@ -107,9 +107,10 @@ bgmv_expand_kernel(Problem p) {
 // covers 64 B rows of the CTA's 256 and every one of its 16-byte loads reads
 // 512 contiguous bytes: K/8 threads share a row, each taking one 16-byte chunk
 // (eight ranks), and the row's sum is completed with shuffles.  The 256 sums
-// go through shared memory to coalesced output stores.  (Two token rows per CTA
-// step, with both rows' loads in flight, measured slower: the register cost
-// halves the CTAs an SM holds.)
+// go through shared memory to coalesced output stores; in add mode the old
+// values of the thread's two output columns are loaded with the B rows, before
+// any of them is used.  (Two token rows per CTA step, with both rows' loads in
+// flight, measured slower: the register cost halves the CTAs an SM holds.)
 template <int OUT_DT, bool ADD>
 __global__ void __launch_bounds__(BGMV_THREADS)
 bgmv_coalesced_kernel(Problem p) {
@@ -129,6 +130,15 @@ bgmv_coalesced_kernel(Problem p) {
     for (int64_t b = blockIdx.y; b < p.batches; b += gridDim.y) {
         const int64_t a = load_meta(p.idx, b);
         if (a < 0 || a >= p.lora_num || b >= lim) continue;     // uniform across the CTA
+        const int64_t oi = b * p.H + p.off + n0;
+        float old[2] = {0.f, 0.f};   // add mode: the old values of columns tid and tid + BGMV_THREADS
+        if (ADD) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = tid + h * BGMV_THREADS;
+                if (n0 + c < p.N) old[h] = load_elem(p.out, OUT_DT, oi + c);
+            }
+        }
         // this thread's eight ranks of x, rounded to B's dtype
         float xv[8];
 #pragma unroll
@@ -162,11 +172,12 @@ bgmv_coalesced_kernel(Problem p) {
             }
         }
         __syncthreads();
-        const int64_t oi = b * p.H + p.off + n0;
-        for (int c = tid; c < BGMV_COLS; c += BGMV_THREADS) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = tid + h * BGMV_THREADS;
             if (n0 + c >= p.N) break;
             const float v = res[c];
-            store_elem(p.out, OUT_DT, oi + c, ADD ? load_elem(p.out, OUT_DT, oi + c) + v : v);
+            store_elem(p.out, OUT_DT, oi + c, ADD ? old[h] + v : v);
         }
         __syncthreads();   // res is read before the next row overwrites it
     }

@@ -309,8 +309,13 @@ struct Plan {
 // chunk count): the one that minimises the bytes the busiest SM moves, i.e.
 // ceil(items / SMs) items of 128 x H/splits x 2 bytes of x, plus its share
 // of the partial sums written and read back (2 x splits x rows x rank x 4
-// bytes over all SMs).  The block count is estimated from the row count and
-// the number of segments (each adds at most one partial block).
+// bytes over all SMs), plus ITEM_FIXED_BYTES per item: each item refills the
+// chunk pipeline and drains its accumulator, about one DRAM latency of one
+// SM's share of the bandwidth.  The block count is estimated from the row
+// count and the number of segments (each adds at most one partial block).
+// Measured on one B200 for hidden 4096 -> rank 16 over 8772 rows (us per
+// call by splits 1/2/4/8/16): 37.4, 24.0, 22.4, 23.8, 25.3; the model picks 4.
+constexpr double ITEM_FIXED_BYTES = 64.0 * 1024.0;
 inline int preferred_splits(const Problem& p, int sm_count) {
     const int64_t t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
     const int64_t blocks = (t_lim + BM - 1) / BM + (p.batches < t_lim ? p.batches : t_lim);
@@ -323,7 +328,7 @@ inline int preferred_splits(const Problem& p, int sm_count) {
         const double items_per_sm = (double)((blocks * s + G - 1) / G);
         const double x_bytes = items_per_sm * BM * (double)cps * CH * 2.0;
         const double partial = s > 1 ? 2.0 * s * (double)t_lim * (double)p.N * 4.0 / (double)G : 0.0;
-        const double cost = x_bytes + partial;
+        const double cost = x_bytes + partial + items_per_sm * ITEM_FIXED_BYTES;
         if (s == 1 || cost < best_cost * 0.98) {   // more splits only for a clear gain
             best = s;
             best_cost = cost;

@@ -1,0 +1,104 @@
+"""Host-side pieces of bench.py: the algorithmic byte count the roofline divides
+by, and the rule that a recorded DRAM figure is used only for the kernel source
+it was taken on.  No GPU is touched."""
+import dataclasses
+import json
+import os
+
+import numpy as np
+import pytest
+
+import bench
+import sgmv_inputs as gen
+
+
+def test_tiny_call_bytes_by_hand():
+    # segments of 4, 6 and 7 rows have adapters 0, 2 and 1; the 3-row one is -1.
+    # Overwrite: x read (16 x 2 B), the slice written (128 x 2 B), three B tiles
+    # of 128 x 16 x 2 B, and three int64 metadata vectors of 4 entries.
+    p = gen.tiny()
+    byts, flops, rows = bench.call_accounting(p, 0)
+    assert rows == 17
+    assert byts == 17 * (16 * 2 + 128 * 2) + 3 * 128 * 16 * 2 + 3 * 4 * 8
+    assert flops == 2 * 128 * 16 * 17
+
+
+def test_add_mode_reads_the_old_slice_too():
+    p = gen.qkv_prefill()
+    q = dataclasses.replace(p, add_inputs=not p.add_inputs)
+    (b_add, _, rows), (b_over, _, _) = (bench.call_accounting(p, 0), bench.call_accounting(q, 0))
+    if not p.add_inputs:
+        b_add, b_over = b_over, b_add
+    so = bench.DT_SIZE[p.out_dt]
+    assert b_add - b_over == rows * p.calls[0].slice_size * so
+
+
+def test_inactive_and_out_of_range_adapters_move_nothing():
+    p = gen.tiny()
+    idx = p.lora_idx.copy()
+    idx[:] = [-1, 7, -1, -5]          # 7 and -5 are outside [0, 3)
+    q = dataclasses.replace(p, lora_idx=idx)
+    byts, flops, rows = bench.call_accounting(q, 0)
+    assert rows == 0 and flops == 0
+    assert byts == 3 * 4 * 8          # the metadata is still read
+
+
+def test_step_sums_its_calls():
+    p = gen.qkv_prefill()
+    per_call = [bench.call_accounting(p, c) for c in range(len(p.calls))]
+    assert bench.step_accounting(p) == tuple(sum(v[i] for v in per_call) for i in range(3))
+
+
+def test_every_kernel_family_hashes_existing_sources():
+    csrc = os.path.join(bench.ROOT, "segmented_gather_gemm_expand_b200", "csrc")
+    for family, files in bench.KERNEL_SOURCES.items():
+        assert "common.cuh" in files, family
+        for fn in files:
+            assert os.path.exists(os.path.join(csrc, fn)), (family, fn)
+        h = bench.kernel_source_hash(family)
+        assert len(h) == 16 and h == bench.kernel_source_hash(family)
+    assert bench.kernel_source_hash("tc") != bench.kernel_source_hash("decode")
+
+
+def _fake_root(tmp_path, source_text):
+    csrc = tmp_path / "segmented_gather_gemm_expand_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for files in bench.KERNEL_SOURCES.values():
+        for fn in files:
+            (csrc / fn).write_text(source_text + fn)
+    (tmp_path / "profiles").mkdir()
+    return tmp_path
+
+
+def test_recorded_traffic_only_for_the_source_it_was_taken_on(tmp_path, monkeypatch):
+    root = _fake_root(tmp_path, "v1 ")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    rec = {"qkv_prefill": {"tc": {"dram_bytes_per_launch": 123.0,
+                                  "kernel_source_hash": bench.kernel_source_hash("tc")}}}
+    (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("qkv_prefill", "tc") == 123.0
+    assert bench.recorded_traffic("qkv_prefill", "decode") is None      # no record for that kernel
+    assert bench.recorded_traffic("decode_mix", "tc") is None           # nor for that workload
+    # a change to a file outside the family keeps the record
+    (root / "segmented_gather_gemm_expand_b200" / "csrc" / "bgmv.cuh").write_text("changed")
+    assert bench.recorded_traffic("qkv_prefill", "tc") == 123.0
+    # a change to the kernel's own source drops it
+    (root / "segmented_gather_gemm_expand_b200" / "csrc" / "tc_kernel.cuh").write_text("changed")
+    assert bench.recorded_traffic("qkv_prefill", "tc") is None
+
+
+def test_missing_traffic_file_gives_none(tmp_path, monkeypatch):
+    root = _fake_root(tmp_path, "v1 ")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.recorded_traffic("qkv_prefill", "tc") is None
+
+
+def test_committed_traffic_records_are_well_formed():
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for workload, kernels in d.items():
+        assert workload in gen.WORKLOADS, workload
+        for family, e in kernels.items():
+            assert family in bench.KERNEL_SOURCES, family
+            assert e["dram_bytes_per_launch"] > 0
+            assert len(e["kernel_source_hash"]) == 16
+            assert os.path.exists(os.path.join(bench.ROOT, e["source"].split(" ")[0]))

@@ -238,10 +238,12 @@ SGMV_API int bgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lor
  *   workspace, workspace_bytes  optional DEVICE scratch (16-byte aligned, else
  *             SGMV_ERR_WORKSPACE), owned by the caller and used only by the
  *             work this call enqueues.  With it the tensor-core kernel splits
- *             H so that every SM has work and adds the fp32 partial sums in a
- *             second kernel, in a fixed order (deterministic); without it
- *             (NULL or too small) each row block is one work item.  Calls
- *             that run at the same time need separate workspaces.
+ *             H into up to 16 parts (the count a cost model of the busiest
+ *             SM's bytes and per-item pipeline work prefers, halved until the
+ *             partial sums fit) and adds the fp32 partial sums in a second
+ *             kernel, in a fixed order (deterministic); without it (NULL or
+ *             too small for two parts) each row block is one work item.
+ *             Calls that run at the same time need separate workspaces.
  *
  * The tensor-core path (SGMV_VARIANT_TC) needs x and lora_a in the same half
  * dtype with unit column stride and 16-byte aligned rows, R a multiple of 16

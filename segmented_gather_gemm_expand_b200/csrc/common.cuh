@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "sgmv.h"
 
 namespace sgmv {
@@ -95,6 +97,21 @@ enum : int32_t {
     DEVERR_TIMEOUT_CONVERT = 8,
     DEVERR_SCHEDULE = 16
 };
+
+// Raises a kernel's dynamic shared-memory limit, once per device: the setting
+// belongs to the device's context, so a process that drives several GPUs sets
+// it on each (devices past 63 set it on every call).  `done` holds one bit per
+// device.  Returns false if the runtime refused.
+template <typename Kern>
+inline bool set_smem_limit_once(Kern kern, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (bit && (done.load() & bit)) return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    if (bit) done.fetch_or(bit);
+    return true;
+}
 
 }  // namespace sgmv
 

@@ -411,12 +411,8 @@ inline bool make_plan(const Problem& p, int sm_count, int splits, tc::EncodeTile
 template <int OUT_DT>
 int launch_dt(const Plan& pl, const Problem& p, float* ws, cudaStream_t stream) {
     auto kern = shrink_kernel<OUT_DT>;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT) != cudaSuccess)
-            return SGMV_ERR_CUDA;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!set_smem_limit_once(kern, SMEM_LIMIT, configured)) return SGMV_ERR_CUDA;
     // Both kernels are launched with programmatic stream serialization: each
     // may start its prologue while the kernel before it drains, and waits
     // (griddepcontrol.wait) before it reads global memory.

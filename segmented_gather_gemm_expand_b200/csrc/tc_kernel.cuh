@@ -1152,13 +1152,8 @@ inline bool make_plan(const Problem* ps, int nsl, int sm_count, Plan* out, int f
 template <int OUT_DT, bool ADD, int BN>
 int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
     auto kern = tc_expand_slice_kernel<OUT_DT, ADD, BN>;
-    static std::atomic<bool> configured{false};
-    if (!configured.load()) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_OPTIN - SMEM_STATIC_RESERVE) != cudaSuccess)
-            return SGMV_ERR_CUDA;
-        configured.store(true);
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!set_smem_limit_once(kern, SMEM_OPTIN - SMEM_STATIC_RESERVE, configured)) return SGMV_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)pl.grid);
     cfg.blockDim = dim3(THREADS);

@@ -26,6 +26,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -94,8 +95,8 @@ def measured_peak():
 
 
 # the source files each kernel family is compiled from (its own header, the PTX
-# wrappers and the shared helpers); a recorded DRAM figure stays valid while these
-# are unchanged
+# wrappers and the shared helpers); a recorded DRAM figure stays valid while their
+# code (comments and layout aside) is unchanged
 KERNEL_SOURCES = {
     "tc": ("common.cuh", "tc.cuh", "tc_kernel.cuh", "tc_ptx.cuh"),
     "simt": ("common.cuh", "simt.cuh"),
@@ -104,12 +105,20 @@ KERNEL_SOURCES = {
 }
 
 
+_COMMENTS = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
+def code_only(text):
+    """C++ source without comments, whitespace runs collapsed."""
+    return " ".join(_COMMENTS.sub(" ", text).split())
+
+
 def kernel_source_hash(variant):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "segmented_gather_gemm_expand_b200", "csrc")
     for fn in KERNEL_SOURCES[variant]:
         h.update(fn.encode())
-        h.update(open(os.path.join(csrc, fn), "rb").read())
+        h.update(code_only(open(os.path.join(csrc, fn), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -87,6 +87,23 @@ def test_recorded_traffic_only_for_the_source_it_was_taken_on(tmp_path, monkeypa
     assert bench.recorded_traffic("qkv_prefill", "tc") is None
 
 
+def test_comment_and_layout_edits_keep_the_record(tmp_path, monkeypatch):
+    root = _fake_root(tmp_path, "int v1; ")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    rec = {"qkv_prefill": {"tc": {"dram_bytes_per_launch": 5.0,
+                                  "kernel_source_hash": bench.kernel_source_hash("tc")}}}
+    (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    f = root / "segmented_gather_gemm_expand_b200" / "csrc" / "tc_kernel.cuh"
+    f.write_text("// a new comment\nint   v1;\n/* another\n one */ tc_kernel.cuh")
+    assert bench.recorded_traffic("qkv_prefill", "tc") == 5.0
+    f.write_text("int v2; tc_kernel.cuh")
+    assert bench.recorded_traffic("qkv_prefill", "tc") is None
+
+
+def test_code_only_strips_comments():
+    assert bench.code_only("a; // b\n/* c\n d */ e;") == "a; e;"
+
+
 def test_missing_traffic_file_gives_none(tmp_path, monkeypatch):
     root = _fake_root(tmp_path, "v1 ")
     monkeypatch.setattr(bench, "ROOT", str(root))

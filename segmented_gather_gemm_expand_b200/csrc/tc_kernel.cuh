@@ -1,40 +1,43 @@
 // Tensor-core SGMV expand-slice for sm_100a: tcgen05 MMA with the accumulator
 // in tensor memory, TMA staging of B, x and the output slice.
 //
-// One persistent CTA per SM, 352 threads in warp roles:
+// One persistent CTA per SM, 352 threads in warp roles.  BN, the n-tile width,
+// is 128 or 256 columns (a template parameter); TMEM holds 512 / BN accumulators.
 //
 //   warp 0    producer   TMA: x for each 128-row block of a segment and B[a]'s
-//                        128-column n-tile (K in 64/32/16/8-column boxes with
-//                        the matching swizzle) for each piece.
+//                        BN-row n-tile (K in 64/32/16/8-column boxes with the
+//                        matching swizzle) for each piece.
 //   warp 2    loader     allocates each piece's rows in shared-memory rings (one
 //                        ring of 128-byte rows per 128-byte column chunk, in
 //                        piece order, freed as the epilogue's stores drain) and,
 //                        in add mode, TMA-loads the old output there: whole
 //                        8-row groups as 2-D boxes of 8..128 rows (128-byte
 //                        swizzle), clipped at the slice's last column.
-//   warp 1    MMA        (mixed dtypes only) rounds x to the weights' dtype into
-//                        the MMA operand layout; one elected lane issues
-//                        tcgen05.mma (M=128 rows, N=128 columns, K=16 each)
-//                        into one of four TMEM accumulators.
+//   warp 1    MMA        rounds x to the weights' dtype into the MMA operand
+//                        layout (mixed dtypes), or repeats a short block's rows
+//                        over the operand (see below); one elected lane issues
+//                        tcgen05.mma (M=128 rows, N=BN columns, K=16 each) into
+//                        one of the TMEM accumulators.
 //   warps 3-10 epilogue  two groups of four warps take alternate pieces; warp w
 //                        owns TMEM lanes 32*(w%4).. (32 rows of the piece) and
 //                        all its columns, or, for a piece of at most 64 rows
 //                        (computed once per 32- or 64-lane span), its rows in
 //                        its span and every 2nd or 4th column chunk: tcgen05.ld
-//                        the fp32 sums, add
-//                        the old output (add mode), round once to the output
-//                        dtype, write the tile back in place in shared memory
-//                        and TMA-store its whole 8-row groups; the last < 8
-//                        rows of a segment are stored from registers, so
-//                        nothing outside the segment's rows is written.
+//                        the fp32 sums, add the old output (add mode), round
+//                        once to the output dtype, write the tile back in place
+//                        in shared memory and TMA-store its whole 8-row groups;
+//                        the last < 8 rows of a segment are stored from
+//                        registers, so nothing outside the segment's rows is
+//                        written.
 //
 // Work is expanded on the device.  A piece is (segment, 128-row block of the
-// segment, 128-column n-tile); pieces are ordered with the n-tile fastest, so
-// the x block is staged once and reused across every n-tile.  Every CTA builds
-// the table of segments in shared memory (the guards of sgmv.h applied),
-// weighs each piece as its 8-row groups plus a fixed part (its B tile and the
-// per-piece pipeline work), and takes the pieces that start in its equal share
-// of the total weight.
+// segment, n-tile); pieces are ordered with the n-tile fastest.  Every CTA
+// builds the table of segments in shared memory (the guards of sgmv.h
+// applied) and then, identically in every CTA, either deals the pieces
+// round-robin (when full and partial blocks are mixed) or gives each CTA the
+// pieces that start in its equal share of the total weight (a piece weighs its
+// 8-row groups, at least a floor, plus its B tile), keeping an x block across
+// its n-tiles.
 // Every wait on an mbarrier is bounded; a wait that gives up sets the device
 // error word and makes the CTA leave its loops.
 #pragma once

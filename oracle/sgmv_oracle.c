@@ -33,9 +33,7 @@
  */
 #include <math.h>
 #include <stdint.h>
-#ifndef ORC_MUTANT
-#define ORC_MUTANT 0   /* >0 only in the mutation test: a deliberate bug to be caught by the pins */
-#endif
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -89,7 +87,7 @@ uint16_t orc_encode16(double v, int dt)
     double n = ldexp(x, -qexp);        /* exact: scaling by a power of two */
     double r = floor(n);
     double rem = n - r;
-    if (rem > 0.5 || (rem == 0.5 && (ORC_MUTANT == 8 || fmod(r, 2.0) != 0.0))) r += 1.0;
+    if (rem > 0.5 || (rem == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;   /* ties to even */
     /* r * 2^qexp is the rounded magnitude; r <= 2^(f+1). */
     if (E < emin) {
         /* subnormal grid; r == 2^f means it rounded up to the smallest normal,
@@ -155,24 +153,23 @@ int64_t orc_expand_slice(const void* x, int x_dt, int64_t x_rows, int64_t K, int
 #pragma omp parallel for num_threads(nthreads) reduction(+ : written) schedule(static)
 #endif
         for (int64_t m = 0; m < L; ++m) {
-            const int64_t r = s + m + (ORC_MUTANT == 6);
+            const int64_t r = s + m;
             if (r >= out_rows || r >= x_rows) continue;
+            /* the row of x cast to the weights' dtype (nearest-even) */
+            double* xhat = (double*)malloc((size_t)(K > 0 ? K : 1) * sizeof(double));
+            for (int64_t k = 0; k < K; ++k) xhat[k] = round_to(load_elem(x, x_dt, r * x_rs + k * x_cs), w_dt);
             for (int64_t n = 0; n < N; ++n) {
                 double acc = 0.0;
                 for (int64_t k = 0; k < K; ++k) {
-                    double xv = load_elem(x, x_dt, r * x_rs + k * x_cs);
-                    if (ORC_MUTANT != 4) xv = round_to(xv, w_dt);
-                    const int64_t nn = ORC_MUTANT == 3 ? (n + 1) % N : n;
-                    double wv = load_elem(w, w_dt, a * w_as + nn * w_ns + k * w_ks);
-                    double prod = xv * wv;
-                    if (ORC_MUTANT == 5) prod = round_to(prod, w_dt);
-                    if (ORC_MUTANT == 2) acc -= prod; else acc += prod;
+                    const double wv = load_elem(w, w_dt, a * w_as + n * w_ns + k * w_ks);
+                    acc += xhat[k] * wv;
                 }
-                const int64_t oi = r * H + (ORC_MUTANT == 7 ? 0 : slice_offset) + n;
-                double v = (add && ORC_MUTANT != 1) ? load_elem(out, out_dt, oi) + acc : acc;
+                const int64_t oi = r * H + slice_offset + n;
+                const double v = add ? load_elem(out, out_dt, oi) + acc : acc;
                 if (pre) pre[r * N + n] = v;
                 store_elem(out, out_dt, oi, v);
             }
+            free(xhat);
             written += 1;
         }
     }

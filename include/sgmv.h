@@ -93,7 +93,7 @@ enum {
     SGMV_ERR_SLICE_OVERLAP = -15,    /* two non-empty slices of one call share a column */
     SGMV_ERR_OUT_WIDTH = -16,        /* sgmv_expand / sgmv_shrink: out.shape[1] != lora_b/lora_a.shape[-2] */
     SGMV_ERR_WORKSPACE = -17,        /* sgmv_shrink: workspace not 16-byte aligned */
-    SGMV_ERR_SCRATCH = -18,          /* sgmv_shrink_static_scratch: the call needs more than the static scratch */
+    SGMV_ERR_SCRATCH = -18,          /* reserved (no entry point returns it) */
     SGMV_ERR_CUDA = -20,             /* a CUDA runtime call failed */
     SGMV_ERR_LAUNCH = -21            /* a kernel launch failed */
 };
@@ -270,17 +270,16 @@ SGMV_API int sgmv_shrink(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, c
  * point instead keeps the partial sums in a scratch array that the library
  * itself declares as a file-scope device variable of
  * SGMV_SHRINK_STATIC_SCRATCH_BYTES, which every GPU that loads the library
- * holds until the process exits.  It computes exactly what sgmv_shrink
- * computes with a workspace that fits its preferred split count, and takes the
- * same arguments without the workspace.
+ * holds until the process exits.  It takes sgmv_shrink's arguments without
+ * the workspace and computes exactly (bit for bit) what sgmv_shrink computes
+ * with a workspace of SGMV_SHRINK_STATIC_SCRATCH_BYTES: the preferred H split
+ * count, halved until the partial sums (splits x min(T_x, T_out) x R x 4
+ * bytes) fit, down to one split, which needs no scratch at all.
  *
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and keeps it; make that first call before any
  *     stream capture.  Later calls only read the kept address.
  *   - It allocates nothing and calls no allocating routine.
- *   - A call whose partial sums need more than SGMV_SHRINK_STATIC_SCRATCH_BYTES
- *     (splits x min(T_x, T_out) x R x 4 bytes) returns SGMV_ERR_SCRATCH before
- *     anything is enqueued; sgmv_shrink with a workspace of your own takes it.
  *   - Every call on a device shares the one array, and it keeps whatever the
  *     last call left there: each call writes every partial sum before it reads
  *     it, so nothing needs to start at zero, but two calls whose work overlaps

@@ -192,7 +192,7 @@ int forced_bn(int forced) { return forced == SGMV_VARIANT_TC_WIDE ? 256 : 0; }
 
 // Which variant runs a validated, non-empty call.
 int choose_variant(const Call& c, const DeviceInfo& dev, int forced) {
-    const bool tc_ok = dev.cc_major == 10 && tc_supports(&c.p, 1, forced_bn(forced));
+    const bool tc_ok = dev.cc_major == 10 && tc_supports(&c.p, 1, dev.sm_count, forced_bn(forced));
     if (forced == SGMV_VARIANT_SIMT) return SGMV_VARIANT_SIMT;
     if (forced == SGMV_VARIANT_DECODE) return SGMV_ERR_VARIANT;   // bgmv_expand_slice's kernel only
     if (forced == SGMV_VARIANT_TC || forced == SGMV_VARIANT_TC_WIDE)
@@ -235,7 +235,7 @@ int choose_multi(const Call* calls, int n, const DeviceInfo& dev, int forced, bo
     if (forced != SGMV_VARIANT_SIMT && dev.cc_major == 10) {
         Problem ps[SGMV_MAX_SLICES];
         for (int i = 0; i < n; ++i) ps[i] = calls[i].p;
-        if (tc_supports(ps, n, forced_bn(forced))) {
+        if (tc_supports(ps, n, dev.sm_count, forced_bn(forced))) {
             *fused = true;
             return SGMV_VARIANT_TC;
         }
@@ -456,20 +456,15 @@ int sgmv_shrink_static_scratch(const sgmv_tensor* inputs, const sgmv_tensor* lor
     if (c.empty) return SGMV_OK;
     DeviceInfo dev;
     if ((rc = device_info(&dev))) return rc;
-    const int forced = g_forced_variant.load();
+    // exactly what sgmv_shrink does with a workspace of the static array's
+    // size: the preferred split count, halved until the partial sums fit
     int splits = 1;
-    // the split count sgmv_shrink would use with an unlimited workspace
-    const int v0 = choose_shrink(c, dev, forced, nullptr, 0, &splits);
-    if (v0 < 0) return v0;
-    if (v0 == SGMV_VARIANT_TC) {
-        splits = shr::preferred_splits(c.p, dev.sm_count);
-        if ((uint64_t)shr::workspace_bytes_for(c.p, splits) > (uint64_t)SGMV_SHRINK_STATIC_SCRATCH_BYTES)
-            return SGMV_ERR_SCRATCH;
-    }
     float* scratch = static_scratch(&rc);
     if (!scratch) return rc;
+    const int v = choose_shrink(c, dev, g_forced_variant.load(), scratch, SGMV_SHRINK_STATIC_SCRATCH_BYTES, &splits);
+    if (v < 0) return v;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (v0 == SGMV_VARIANT_TC) return launch_shrink(c, dev, splits, scratch, st);
+    if (v == SGMV_VARIANT_TC) return launch_shrink(c, dev, splits, scratch, st);
     return launch_simt(c, dev, st);
 }
 
@@ -688,7 +683,7 @@ const char* sgmv_status_string(int code) {
         case SGMV_ERR_SLICE_OVERLAP: return "two slices of a multi-slice call overlap";
         case SGMV_ERR_OUT_WIDTH: return "out.shape[1] != lora_b.shape[-2] (plain expand and shrink write whole rows)";
         case SGMV_ERR_WORKSPACE: return "workspace is not 16-byte aligned";
-        case SGMV_ERR_SCRATCH: return "the call needs more scratch than sgmv_shrink_static_scratch's static array holds";
+        case SGMV_ERR_SCRATCH: return "reserved status (no entry point returns it)";
         case SGMV_ERR_CUDA: return "a CUDA runtime call failed";
         case SGMV_ERR_LAUNCH: return "kernel launch failed";
         default: return "unknown status";

@@ -1173,9 +1173,9 @@ int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
 
 }  // namespace tc
 
-bool tc_supports(const Problem* ps, int nsl, int force_bn) {
+bool tc_supports(const Problem* ps, int nsl, int sm_count, int force_bn) {
     tc::Plan pl;
-    return tc::make_plan(ps, nsl, 148, &pl, force_bn);
+    return tc::make_plan(ps, nsl, sm_count, &pl, force_bn);
 }
 
 template <int BN>

@@ -147,3 +147,60 @@ def run_multi(dp: DeviceProblem, calls=None, out=None, plan_only=False):
     y = dp.y if out is None else out
     fn = sg.plan_multi_slice if plan_only else sg.sgmv_expand_multi_slice
     return fn(dp.x, ws, y, dp.start, dp.len, dp.idx, p.batches, p.max_seq_len, offs, p.add_inputs)
+
+
+def _bits(a: np.ndarray) -> np.ndarray:
+    """The storage's bit patterns (so that NaNs compare by their bits)."""
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def compare_every_element(gpu: np.ndarray, ref: np.ndarray, p: gen.Problem, regs, chunk_rows: int = 1024):
+    """Compare a whole output with the oracle's, element by element, in row chunks.
+
+    regs: [(rows_mask, col0, ncols), ...], the written regions.  Inside them every
+    element must be within the stated tolerance of the oracle's value; every
+    other element must keep the bits of p.y0.  Returns (max |err|, elements
+    compared inside the regions).
+    """
+    dt = p.out_dt
+    T, H = gpu.shape
+    worst, count = 0.0, 0
+    for r0 in range(0, T, chunk_rows):
+        r1 = min(T, r0 + chunk_rows)
+        g, rf, y0 = gpu[r0:r1], ref[r0:r1], p.y0[r0:r1]
+        outside = np.ones(g.shape, dtype=bool)
+        for rows, c0, n in regs:
+            outside[np.ix_(rows[r0:r1], np.arange(c0, c0 + n))] = False
+        bad = np.nonzero((_bits(g) != _bits(y0)) & outside)
+        assert bad[0].size == 0, (f"{bad[0].size} untouched elements changed, first at row "
+                                  f"{r0 + bad[0][0]}, column {bad[1][0]}")
+        for rows, c0, n in regs:
+            sel = rows[r0:r1]
+            if not sel.any():
+                continue
+            gv = decode(g[sel, c0:c0 + n], dt)
+            rv = decode(rf[sel, c0:c0 + n], dt)
+            special = (np.isnan(gv) & np.isnan(rv)) | (np.isinf(gv) & np.isinf(rv) & (np.sign(gv) == np.sign(rv)))
+            fin = ~special
+            assert np.array_equal(np.isfinite(gv[fin]), np.isfinite(rv[fin])), f"non-finite mismatch in rows {r0}..{r1}"
+            err = np.abs(gv[fin] - rv[fin])
+            tol = tolerance(rv[fin], dt, p.rank)
+            if err.size:
+                i = np.argmax(err - tol)
+                assert err[i] <= tol[i], (f"rows {r0}..{r1}: err {err[i]:.3g} > tol {tol[i]:.3g} "
+                                          f"(gpu {gv[fin][i]!r}, oracle {rv[fin][i]!r})")
+                worst = max(worst, float(err.max()))
+            count += int(gv.size)
+    return worst, count
+
+
+def report(name: str, **fields):
+    """Print a parity record, and append it as a JSON line to $SGMV_PARITY_REPORT if set."""
+    import json
+    import os
+    rec = dict(test=name, **fields)
+    print(json.dumps(rec))
+    path = os.environ.get("SGMV_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")

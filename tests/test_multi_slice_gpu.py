@@ -134,19 +134,6 @@ def test_empty_slice_is_skipped():
     assert np.array_equal(gm, gs)
 
 
-@pytest.mark.parametrize("name", ["qkv_prefill", "mlp_mixed"])
-def test_workload_fused_equals_single_calls(name):
-    """The bench workloads with several slices: one fused call == the separate calls, bit for bit."""
-    p = gen.WORKLOADS[name]()
-    dm = DeviceProblem(p)
-    assert run_multi(dm, plan_only=True) == (sg.VARIANT_TC, 1)
-    run_multi(dm)
-    torch.cuda.synchronize()
-    gm = dm.result()
-    del dm
-    ds = DeviceProblem(p)
-    for c in range(len(p.calls)):
-        ds.run(c)
-    torch.cuda.synchronize()
-    assert sg.device_error() == 0
-    assert np.array_equal(gm, ds.result())
+# The full-size workloads of several slices (QKV prefill, gate/up MLP) run through the fused
+# launch in test_parity_gpu.test_workload_full_size_every_element, against the oracle at every
+# element and against the separate calls bit for bit.

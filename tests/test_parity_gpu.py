@@ -11,7 +11,8 @@ import torch
 import oracle
 import sgmv_inputs as gen
 import segmented_gather_gemm_expand_b200 as sg
-from sgmv_testlib import DeviceProblem, compare, from_torch, to_torch, written_rows
+from sgmv_testlib import (DeviceProblem, compare, compare_every_element, from_torch, report, run_multi,
+                          to_torch, written_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -269,53 +270,107 @@ def test_add_equals_old_plus_overwrite_result(variant):
 
 # ------------------------------------------------------------------ the five workloads, full size
 
-def sampled_subproblem(p: gen.Problem, rng, n_segments: int, cap: int):
-    """Segments chosen by `rng`; from each, its first and last `cap` rows."""
-    A = p.calls[0].w.shape[0]
-    valid = [b for b in range(p.batches) if 0 <= p.lora_idx[b] < A and p.seq_len[b] > 0]
-    pick = sorted(set([valid[0], valid[-1]] + list(rng.choice(valid, size=min(n_segments, len(valid)),
-                                                               replace=False))))
-    starts, lens, idx = [], [], []
-    for b in pick:
-        s, L, a = int(p.seq_start[b]), int(p.seq_len[b]), int(p.lora_idx[b])
-        if L <= 2 * cap:
-            starts.append(s), lens.append(L), idx.append(a)
-        else:
-            starts += [s, s + L - cap]
-            lens += [cap, cap]
-            idx += [a, a]
-    return np.array(starts, np.int64), np.array(lens, np.int64), np.array(idx, np.int64)
-
-
-@pytest.mark.parametrize("variant", VARIANTS)
-@pytest.mark.parametrize("name", ["qkv_prefill", "mlp_mixed", "long_single", "decode_mix"])
-def test_workload_full_size(name, variant):
-    p = gen.WORKLOADS[name]()
-    dp = DeviceProblem(p)
-    if not use_variant(variant, dp):
-        pytest.skip("variant does not take this case")
-    for c in range(len(p.calls)):
-        dp.run(c)
-    torch.cuda.synchronize()
-    assert sg.device_error() == 0
-    gpu = dp.result()
-    del dp
-    torch.cuda.empty_cache()
-    s, l, i = sampled_subproblem(p, np.random.default_rng(5), 6, 40)
-    sub = gen.Problem(p.name, p.x, p.x_dt, p.w_dt, p.y0, p.out_dt, s, l, i, p.add_inputs, p.calls)
+def oracle_all_calls(p):
     ref = p.y0
     for c in range(len(p.calls)):
-        ref = oracle.run_problem(sub, out=ref, call=c, nthreads=oracle.max_threads())
-    check_rows = written_rows(sub)
-    check_regions(gpu, ref, p, regions(p), check_rows=check_rows)
+        ref = oracle.run_problem(p, out=ref, call=c, nthreads=oracle.max_threads())
+    return ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "qkv_prefill", "mlp_mixed", "long_single", "decode_mix"])
+def test_workload_full_size_every_element(name):
+    """Every written element of every slice of the workload against the oracle (the multi-threaded C
+    oracle computes the whole output once); every other element bit-exact.  Each variant that takes
+    the case runs it, and for workloads of several slices so does the fused multi-slice launch, which
+    must also equal the separate calls bit for bit."""
+    p = gen.WORKLOADS[name]()
+    ref = oracle_all_calls(p)
+    regs = regions(p)
+    expected = int(sum(int(rows.sum()) * n for rows, _, n in regs))
+    single = {}
+    for variant in VARIANTS:
+        dp = DeviceProblem(p)
+        if not use_variant(variant, dp):
+            report(f"{name}/{variant}", skipped="variant does not take this case")
+            continue
+        for c in range(len(p.calls)):
+            dp.run(c)
+        torch.cuda.synchronize()
+        assert sg.device_error() == 0
+        gpu = dp.result()
+        del dp
+        torch.cuda.empty_cache()
+        sg.set_variant(sg.VARIANT_AUTO)
+        err, count = compare_every_element(gpu, ref, p, regs)
+        assert count == expected, (count, expected)
+        report(f"{name}/{variant}", compared=count, max_abs_err=err, out_dtype=p.out_dt, rank=p.rank)
+        single[variant] = gpu
+    if len(p.calls) > 1:
+        dm = DeviceProblem(p)
+        assert run_multi(dm, plan_only=True) == (sg.VARIANT_TC, 1)
+        run_multi(dm)
+        torch.cuda.synchronize()
+        assert sg.device_error() == 0
+        gm = dm.result()
+        del dm
+        torch.cuda.empty_cache()
+        err, count = compare_every_element(gm, ref, p, regs)
+        assert count == expected, (count, expected)
+        report(f"{name}/fused_multi_slice", compared=count, max_abs_err=err, out_dtype=p.out_dt, rank=p.rank)
+        # the library's automatic choice for the separate calls is the tensor-core kernel (checked below)
+        assert np.array_equal(gm, single["tc"]), "fused launch differs from the separate tensor-core calls"
 
 
 def test_auto_picks_tensor_cores_for_the_workloads():
-    for name in ["qkv_prefill", "decode_mix", "long_single"]:
+    """On compute capability 10.x every workload's calls take the tensor-core kernel."""
+    major, _ = torch.cuda.get_device_capability()
+    assert major == 10, "the tensor-core kernel is built for sm_100a"
+    sg.set_variant(sg.VARIANT_AUTO)
+    for name in ["tiny", "qkv_prefill", "mlp_mixed", "long_single", "decode_mix"]:
         p = gen.WORKLOADS[name]()
-        p.y0 = p.y0[:8]                        # planning needs shapes only
         dp = DeviceProblem(p)
-        assert dp.plan() in (sg.VARIANT_SIMT, sg.VARIANT_TC)
+        for c in range(len(p.calls)):
+            assert dp.plan(c) == sg.VARIANT_TC, (name, c)
+        if len(p.calls) > 1:
+            assert run_multi(dp, plan_only=True) == (sg.VARIANT_TC, 1), name
+
+
+# Each CTA of the tensor-core kernel handles more pieces than its output ring has
+# barrier slots (32), so ring space and barrier phases are reused many times over,
+# in both ways of handing out pieces.  The oracle checks every element.
+MANY_PIECES = {
+    # almost all blocks partial: contiguous ranges
+    "contiguous": dict(short_share=1.0),
+    # 40 % partial blocks: round-robin
+    "round_robin": dict(short_share=0.4),
+}
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("case", sorted(MANY_PIECES))
+def test_more_pieces_per_cta_than_ring_slots(case, variant):
+    rng = np.random.default_rng(77 if case == "contiguous" else 78)
+    B = 1000
+    short = rng.random(B) < MANY_PIECES[case]["short_share"]
+    lengths = np.where(short, rng.integers(1, 128, B), 128)
+    idx = rng.integers(-1, 8, B)
+    N = 1280                           # 10 n-tiles of 128 columns, 5 of 256
+    p = gen.custom(seed=79, lengths=lengths.tolist(), K=16, N=N, H=N + 256, offset=128, num_adapters=8,
+                   idx=idx.tolist())
+    dp = DeviceProblem(p)
+    if not use_variant(variant, dp):
+        pytest.skip(f"{variant} does not take this case")
+    dp.run()
+    torch.cuda.synchronize()
+    assert sg.device_error() == 0
+    gpu = dp.result()
+    ref = oracle.run_problem(p, nthreads=oracle.max_threads())
+    err, count = compare_every_element(gpu, ref, p, regions(p))
+    active = (p.lora_idx >= 0) & (p.lora_idx < 8)
+    pieces = int((np.ceil(lengths[active] / 128) * (N // (256 if variant == "tc_wide" else 128))).sum())
+    report(f"many_pieces_{case}/{variant}", compared=count, max_abs_err=err,
+           pieces_per_cta=pieces / torch.cuda.get_device_properties(0).multi_processor_count)
+    assert pieces > 32 * torch.cuda.get_device_properties(0).multi_processor_count
 
 
 # ------------------------------------------------------------------ metadata validation

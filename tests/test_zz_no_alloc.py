@@ -3,13 +3,18 @@
 Some callers may not allocate device memory at all (a runtime that reserves
 the whole GPU up front, a plugin host that only passes buffers in and out, a
 serving loop that must not stall on cudaMalloc).  This entry point keeps the
-shrink's partial sums in scratch the library declares itself, so such a
-caller gets the same result as sgmv_shrink with a workspace of its own.  The
-test calls it through the C ABI twice in a row, on different inputs, and
-checks each result against sgmv_shrink's within the tolerance the other tests
-use; it also checks that a call needing more scratch than the library holds is
-refused before anything is written.  It lives in a file of its own, collected
-last, and passes alone in a fresh process or after the other tests.
+shrink's split-H partial sums in scratch the library declares itself, so such
+a caller gets exactly what sgmv_shrink computes with a workspace of the same
+size (SGMV_SHRINK_STATIC_SCRATCH_BYTES, 8 MiB).
+
+The test calls it through the C ABI twice in a row, on different inputs, and
+checks each result bit for bit against sgmv_shrink given an 8 MiB workspace of
+its own (same split count, same fixed-order reduction), and every element
+against the CPU oracle's shrink within the tolerance the other tests use.  The
+inputs include a segment with adapter -1 and one of length zero, whose rows
+must keep their bits.  A call whose preferred split count needs more than
+8 MiB of partial sums runs with fewer splits, as sgmv_shrink does.  The file
+is collected last and passes alone in a fresh process or after the other tests.
 """
 import ctypes
 
@@ -17,17 +22,20 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import sgmv_inputs as gen
 import segmented_gather_gemm_expand_b200 as sg
 from segmented_gather_gemm_expand_b200 import _abi
-from sgmv_testlib import compare, from_torch, to_torch
+from sgmv_testlib import compare_every_element, from_torch, report, to_torch
 
 pytestmark = pytest.mark.gpu
 
+STATIC_BYTES = 8 << 20          # SGMV_SHRINK_STATIC_SCRATCH_BYTES in include/sgmv.h
 
-def shrink_problem(seed, lengths, H, R, A, out_dt):
+
+def shrink_problem(seed, lengths, H, R, A, out_dt, idx=None):
     return gen.custom(seed=seed, lengths=lengths, K=H, N=R, H=R, offset=0, num_adapters=A, add_inputs=False,
-                      out_dt=out_dt)
+                      out_dt=out_dt, idx=idx)
 
 
 def device_args(p):
@@ -38,7 +46,7 @@ def device_args(p):
 
 
 def static_scratch_call(x, a, y, meta, p):
-    """The new entry point, called through the C ABI with ctypes."""
+    """The entry point under test, called through the C ABI with ctypes."""
     d = [sg._desc(t) for t in (x, a, y, *meta)]
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return sg._lib.sgmv_shrink_static_scratch(*[ctypes.byref(t) for t in d], p.batches, p.max_seq_len, stream)
@@ -52,40 +60,54 @@ def written_rows(p):
     return rows
 
 
-@pytest.mark.parametrize("case", [0, 1])
-def test_two_calls_in_a_row_match_the_workspace_entry_point(case):
+def oracle_shrink(p):
+    return oracle.shrink(p.x, p.x_dt, p.calls[0].w, p.w_dt, p.y0, p.out_dt, p.seq_start, p.seq_len, p.lora_idx,
+                         nthreads=oracle.max_threads())
+
+
+def check_one(p, name):
+    x, a, y, meta = device_args(p)
+    v, splits, _ = sg.shrink_plan(x, a, y, *meta, p.batches, p.max_seq_len, STATIC_BYTES)
+    ws = torch.empty(STATIC_BYTES, dtype=torch.uint8, device="cuda")
+    y_ref = y.clone()
+    sg.sgmv_shrink(x, a, y_ref, *meta, p.batches, p.max_seq_len, workspace=ws)
+    rc = static_scratch_call(x, a, y, meta, p)
+    assert rc == 0, _abi.STATUS_NAMES.get(rc, rc)
+    torch.cuda.synchronize()
+    assert sg.device_error() == 0
+    got, want = from_torch(y, p.out_dt), from_torch(y_ref, p.out_dt)
+    assert np.array_equal(got, want), "differs from sgmv_shrink with an 8 MiB workspace"
+    rows = written_rows(p)
+    err, count = compare_every_element(got, oracle_shrink(p), p, [(rows, 0, p.calls[0].w.shape[-2])])
+    assert count == int(rows.sum()) * p.calls[0].w.shape[-2]
+    report(f"static_scratch/{name}", variant=v, splits=splits, compared=count, max_abs_err=err)
+    return v, splits
+
+
+PROBLEMS = {
+    # a -1 segment and a zero-length segment among them: their rows keep their bits
+    "bf16_out": dict(seed=31, lengths=[300, 64, 0, 9, 700, 40], H=2048, R=16, A=4, out_dt="bf16",
+                     idx=[0, -1, 2, 1, 3, 2]),
+    "f32_out": dict(seed=32, lengths=[128, 5, 400, 0], H=1000, R=32, A=3, out_dt="f32", idx=[2, 0, 1, 0]),
+}
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_two_calls_in_a_row_match_the_workspace_entry_point(order):
     sg.set_variant(sg.VARIANT_AUTO)
-    problems = [shrink_problem(31, [300, 64, 9, 700], H=2048, R=16, A=4, out_dt="bf16"),
-                shrink_problem(32, [128, 5, 400], H=1000, R=32, A=3, out_dt="f32")]
-    if case:
-        problems.reverse()
-    for p in problems:                      # two calls in a row on one device
-        x, a, y, meta = device_args(p)
-        v, splits, pref = sg.shrink_plan(x, a, y, *meta, p.batches, p.max_seq_len, 1 << 30)
+    names = sorted(PROBLEMS)
+    if order:
+        names.reverse()
+    for name in names:                      # two calls in a row on one device
+        v, splits = check_one(shrink_problem(**PROBLEMS[name]), name)
         assert v == sg.VARIANT_TC and splits > 1
-        assert pref <= _abi_static_bytes()
-        ws = torch.empty(pref, dtype=torch.uint8, device="cuda")
-        y_ref = y.clone()
-        sg.sgmv_shrink(x, a, y_ref, *meta, p.batches, p.max_seq_len, workspace=ws)
-        rc = static_scratch_call(x, a, y, meta, p)
-        assert rc == 0, _abi.STATUS_NAMES.get(rc, rc)
-        torch.cuda.synchronize()
-        assert sg.device_error() == 0
-        compare(from_torch(y, p.out_dt), from_torch(y_ref, p.out_dt), p.y0, p, written_rows(p), 0,
-                p.calls[0].w.shape[-2])
 
 
-def test_a_call_needing_more_scratch_is_refused():
+def test_a_call_whose_preferred_splits_do_not_fit_runs_with_fewer():
     sg.set_variant(sg.VARIANT_AUTO)
     p = shrink_problem(33, [2100], H=4096, R=128, A=1, out_dt="f32")   # splits x 2100 rows x 128 x 4 B > 8 MiB
     x, a, y, meta = device_args(p)
-    _, splits, pref = sg.shrink_plan(x, a, y, *meta, p.batches, p.max_seq_len, 1 << 40)
-    assert pref > _abi_static_bytes(), (splits, pref)
-    rc = static_scratch_call(x, a, y, meta, p)
-    assert rc == _abi.STATUS["SGMV_ERR_SCRATCH"]
-    torch.cuda.synchronize()
-    assert np.array_equal(from_torch(y, p.out_dt), p.y0)
-
-
-def _abi_static_bytes():
-    return 8 << 20          # SGMV_SHRINK_STATIC_SCRATCH_BYTES in include/sgmv.h
+    _, pref_splits, pref = sg.shrink_plan(x, a, y, *meta, p.batches, p.max_seq_len, 1 << 40)
+    assert pref > STATIC_BYTES, (pref_splits, pref)
+    v, splits = check_one(p, "preferred_splits_too_large")
+    assert v == sg.VARIANT_TC and splits < pref_splits

@@ -15,10 +15,14 @@ region and bracketed by a barrier and a device synchronise on both sides; max
 over ranks.  The kernel's average launch duration is the region time divided
 by the launches in it (kernels run back to back; gaps between them count).  The output (215 MB
 for the default workload) is larger than L2 and every step streams all of it,
-so no flush is needed between steps.  `value` is algorithmic HBM bytes of all
-ranks / time; `e2e` repeats the measurement through the same C-ABI calls with
-the inputs in pinned host memory, copying them in and the output back every
-step.  `--impl reference` times the CPU oracle on host cores instead (rank 0).
+so no flush is needed between steps; `l2_flushed` reports the median of 60
+steps with a 256 MiB write before each, to show it.  `eager` times 100 steps
+of plain calls without a graph and the host time inside each call.  `value`
+is algorithmic HBM bytes of all ranks / time; `configs` holds the same
+figures for each of the five expand-slice workloads (their own inputs);
+`e2e` repeats the measurement through the same C-ABI calls with the inputs in
+pinned host memory, copying them in and the output back every step.
+`--impl reference` times the CPU oracle on host cores instead (rank 0).
 """
 import argparse
 import ctypes
@@ -59,6 +63,9 @@ WORKLOAD_TEXT = {
 }
 
 DT_SIZE = {"f16": 2, "bf16": 2, "f32": 4}
+
+# the five expand-slice workloads every default run reports (the `configs` key)
+CONFIG_WORKLOADS = ("tiny", "qkv_prefill", "mlp_mixed", "long_single", "decode_mix")
 
 
 # ---------------------------------------------------------------- accounting
@@ -122,17 +129,30 @@ def kernel_source_hash(variant):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, variant):
-    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+def _traffic_entry(workload, variant):
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         d = json.load(open(path))
         e = d[workload][variant]
         if e.get("kernel_source_hash") == kernel_source_hash(variant):
-            return float(e["dram_bytes_per_launch"])
+            return e
     except Exception:
         pass
     return None
+
+
+def recorded_traffic(workload, variant):
+    """DRAM bytes (read + write) per launch from a committed ncu summary, if taken on the current kernel source."""
+    e = _traffic_entry(workload, variant)
+    return float(e["dram_read_bytes_per_launch"] + e["dram_write_bytes_per_launch"]) if e else None
+
+
+def recorded_traffic_split(workload, variant):
+    e = _traffic_entry(workload, variant)
+    if not e:
+        return None
+    rd, wr = float(e["dram_read_bytes_per_launch"]), float(e["dram_write_bytes_per_launch"])
+    return {"traffic": rd + wr, "read": rd, "write": wr}
 
 
 # ---------------------------------------------------------------- ranks
@@ -295,73 +315,176 @@ def time_graph_region(step, steps, stream, torch):
 
 # ---------------------------------------------------------------- our arm
 
+SECONDARY_STEPS = 200        # graph-replayed steps for each extra config (at least)
+FLUSH_BYTES = 256 << 20      # the L2 flush between steps of the flushed timing
+FLUSH_STEPS = 60             # steps of the flushed timing (median reported)
+EAGER_STEPS = 100            # steps of the eager (no graph) timing
+
+
+def workload_config(p, name, world, step_fused=False):
+    """The `config` object of a bench line: the workload, identical in both arms."""
+    _, _, rows = step_accounting(p)
+    ncalls = len(p.calls)
+    out_mb = p.y0.size * DT_SIZE[p.out_dt] / 1e6
+    return {"workload": WORKLOAD_TEXT[name], "name": name,
+            "batches": p.batches, "tokens_per_rank": p.total_tokens,
+            "active_tokens_per_rank": rows // max(ncalls, 1), "rank": p.rank,
+            "slices": ncalls, "slice_size": p.calls[0].slice_size,
+            "adapters": int(p.calls[0].w.shape[0]), "add_inputs": bool(p.add_inputs),
+            "x_dtype": p.x_dt, "w_dtype": p.w_dt, "out_dtype": p.out_dt,
+            "parallelism": f"replicas x{world} (independent batches, no collective)",
+            "l2": f"no flush between steps: every step streams the whole {out_mb:.0f} MB output, larger than L2 "
+                  f"(a flushed median is reported beside it)",
+            "seed": p.seed,
+            "step": ("all slices in one sgmv_expand_multi_slice call" if step_fused else
+                     f"{ncalls} separate call(s)")}
+
+
+class Resident:
+    """A workload's inputs resident in HBM, with its C-ABI calls pre-marshalled."""
+
+    def __init__(self, p, device):
+        import torch
+        import segmented_gather_gemm_expand_b200 as sg
+        self.p = p
+        tdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+        def host_tensor(a, dt):
+            t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if dt != "f32" else np.ascontiguousarray(a))
+            return t.view(tdt[dt]) if dt != "f32" else t
+
+        self.hx = host_tensor(p.x, p.x_dt)
+        self.hws = [host_tensor(c.w, p.w_dt) for c in p.calls]
+        self.hy = host_tensor(p.y0, p.out_dt)
+        self.hmeta = [torch.from_numpy(a.astype(np.int64)) for a in (p.seq_start, p.seq_len, p.lora_idx)]
+        self.x = self.hx.to(device)
+        self.ws = [w.to(device) for w in self.hws]
+        self.y = self.hy.to(device)
+        self.meta = [m.to(device) for m in self.hmeta]
+        self.workspace = None
+        x, ws, y, meta = self.x, self.ws, self.y, self.meta
+        if p.op == "shrink":
+            _, _, pref = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, 1 << 34)
+            self.workspace = torch.empty(max(pref, 16), dtype=torch.uint8, device=device)
+        self.run, _ = make_calls(p, (x, ws, y, meta), None, None, workspace=self.workspace)
+        self.ncalls = len(p.calls)
+        self.shrink_splits = 0
+        if p.op == "shrink":
+            v_used, self.shrink_splits, _ = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len,
+                                                           self.workspace.numel())
+        elif p.op == "bgmv":
+            v_used = sg.bgmv_plan(x, ws[0], y, meta[2], p.calls[0].slice_offset, p.calls[0].slice_size,
+                                  p.add_inputs)
+        else:
+            v_used = sg.plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, p.calls[0].slice_offset,
+                             p.calls[0].slice_size, p.add_inputs)
+        self.variant = {1: "simt", 2: "tc", 3: "decode"}.get(v_used, str(v_used))
+        # which kernel family's source a recorded DRAM figure must match
+        self.kernel_family = "shrink" if (p.op == "shrink" and self.variant == "tc") else self.variant
+        # kernel launches one call makes (a split shrink adds the partial-sum reduction)
+        self.launches_per_call = 2 if (p.op == "shrink" and self.shrink_splits > 1) else 1
+
+    def step(self, st):
+        for c in range(self.ncalls):
+            self.run(c, st)
+
+    def multi_call(self):
+        return make_multi_call(self.p, (self.x, self.ws, self.y, self.meta))
+
+
+def warm(step, n, stream, torch):
+    with torch.cuda.stream(stream):
+        for _ in range(n):
+            step(stream.cuda_stream)
+    torch.cuda.synchronize()
+
+
+def time_flushed(step, steps, stream, torch, device):
+    """Per-step device time with a FLUSH_BYTES write (larger than L2) before every step;
+    events bracket the step alone.  Returns the list of per-step milliseconds."""
+    buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            buf.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step(stream.cuda_stream)
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    out = [a.elapsed_time(b) for a, b in ev]
+    del buf
+    return out
+
+
+def time_eager(step, steps, stream, torch):
+    """Back-to-back eager calls (no graph): device time of the region, and host
+    time spent inside the calls (argument checks, planning, tensor maps, launch)."""
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        h0 = time.perf_counter()
+        for _ in range(steps):
+            step(stream.cuda_stream)
+        h1 = time.perf_counter()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1), (h1 - h0) * 1e3
+
+
+def secondary_entry(name, seed, steps, warmup, device, peak):
+    """Graph-timed figures of one more workload (its own inputs, freed afterwards)."""
+    import torch
+    import segmented_gather_gemm_expand_b200 as sg
+    p = gen.WORKLOADS[name](seed=seed)
+    r = Resident(p, device)
+    stream = torch.cuda.Stream(device)
+    warm(r.step, warmup, stream, torch)
+    ms = time_graph_region(r.step, steps, stream, torch)
+    assert sg.device_error(device) == 0, "a kernel reported a device-side error"
+    b, f, rows = step_accounting(p)
+    ncalls = r.ncalls
+    us_call = ms * 1e3 / (steps * ncalls)
+    call_bytes = b / ncalls
+    entry = {"workload": WORKLOAD_TEXT[name], "variant": r.variant, "calls_per_step": ncalls,
+             "us_per_call": us_call, "gb_s": call_bytes / (us_call * 1e-6) / 1e9,
+             "frac": call_bytes / (us_call * 1e-6) / 1e9 / peak,
+             "tokens_per_s": p.total_tokens * steps / (ms * 1e-3),
+             "tflops": f * steps / (ms * 1e-3) / 1e12, "bytes_per_call": call_bytes, "steps": steps,
+             "traffic": recorded_traffic(name, r.kernel_family)}
+    del r
+    torch.cuda.empty_cache()
+    return entry
+
+
 def bench_ours(args, rank, world, device):
     import torch
     import segmented_gather_gemm_expand_b200 as sg
-    from segmented_gather_gemm_expand_b200 import _abi
 
     torch.cuda.set_device(device)
     variants = {"auto": sg.VARIANT_AUTO, "simt": sg.VARIANT_SIMT, "tc": sg.VARIANT_TC}
     sg.set_variant(variants[args.variant])
     p = gen.WORKLOADS[args.workload](seed=args.seed + rank)
-    tdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
-
-    def host_tensor(a, dt):
-        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if dt != "f32" else np.ascontiguousarray(a))
-        return t.view(tdt[dt]) if dt != "f32" else t
-
-    hx = host_tensor(p.x, p.x_dt)
-    hws = [host_tensor(c.w, p.w_dt) for c in p.calls]
-    hy = host_tensor(p.y0, p.out_dt)
-    hmeta = [torch.from_numpy(a.astype(np.int64)) for a in (p.seq_start, p.seq_len, p.lora_idx)]
-    x = hx.to(device)
-    ws = [w.to(device) for w in hws]
-    y = hy.to(device)
-    meta = [m.to(device) for m in hmeta]
-    workspace = None
-    if p.op == "shrink":
-        _, _, pref = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, 1 << 34)
-        workspace = torch.empty(max(pref, 16), dtype=torch.uint8, device=device)
-    run, _ = make_calls(p, (x, ws, y, meta), _abi, None, workspace=workspace)
-    ncalls = len(p.calls)
-    shrink_splits = 0
-    if p.op == "shrink":
-        v_used, shrink_splits, _ = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len,
-                                                  workspace.numel())
-    elif p.op == "bgmv":
-        v_used = sg.bgmv_plan(x, ws[0], y, meta[2], p.calls[0].slice_offset, p.calls[0].slice_size,
-                              p.add_inputs)
-    else:
-        v_used = sg.plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, p.calls[0].slice_offset,
-                         p.calls[0].slice_size, p.add_inputs)
-    variant_name = {1: "simt", 2: "tc", 3: "decode"}.get(v_used, str(v_used))
-    # which kernel family's source a recorded DRAM figure must match
-    kernel_family = "shrink" if (p.op == "shrink" and variant_name == "tc") else variant_name
-    # kernel launches one call makes (a split shrink adds the partial-sum reduction)
-    launches_per_call = 2 if (p.op == "shrink" and shrink_splits > 1) else 1
+    r = Resident(p, device)
+    ncalls = r.ncalls
     # One step: the slice calls one by one, or (--step fused) all slices in one
     # sgmv_expand_multi_slice call.
     fused_step = args.step == "fused" and ncalls > 1 and p.op == "slice"
     if fused_step:
-        run_multi_step = make_multi_call(p, (x, ws, y, meta))
-        _, launches_per_step = sg.plan_multi_slice(x, ws, y, *meta, p.batches, p.max_seq_len,
+        run_multi_step = r.multi_call()
+        _, launches_per_step = sg.plan_multi_slice(r.x, r.ws, r.y, *r.meta, p.batches, p.max_seq_len,
                                                    [c.slice_offset for c in p.calls], p.add_inputs)
 
         def step_fn(st):
             run_multi_step(st)
     else:
-        launches_per_step = ncalls * launches_per_call
-
-        def step_fn(st):
-            for c in range(ncalls):
-                run(c, st)
+        launches_per_step = ncalls * r.launches_per_call
+        step_fn = r.step
 
     stream = torch.cuda.Stream(device)
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step_fn(stream.cuda_stream)
-    torch.cuda.synchronize()
+    warm(step_fn, args.warmup, stream, torch)
 
     # Capture the timed steps as graphs of back-to-back launches.
     K = args.steps
@@ -421,12 +544,41 @@ def bench_ours(args, rank, world, device):
     achieved = call_bytes / (avg_launch_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
 
+    # ---- the same step with an L2 flush before every step, median of FLUSH_STEPS
+    flushed = None
+    if not args.no_flush:
+        fl = time_flushed(step_fn, FLUSH_STEPS, stream, torch, device)
+        med = statistics.median(fl)
+        med = reduce_over_ranks(med, 0, 0, 0, device, world)[0]
+        assert sg.device_error(device) == 0, "a kernel reported a device-side error"
+        f_ach = call_bytes / (med / calls_per_step * 1e-3) / 1e9
+        flushed = {"ms_per_step_median": med, "ms_per_step_min": min(fl), "ms_per_step_max": max(fl),
+                   "steps": FLUSH_STEPS, "value": all_bytes / (med * 1e-3) / 1e9, "unit": "GB/s",
+                   "achieved": f_ach, "frac": f_ach / peak,
+                   "note": f"a {FLUSH_BYTES >> 20} MiB write before every step; CUDA events around each step "
+                           f"alone (eager launches, no graph); median over steps"}
+
+    # ---- eager back-to-back steps (no graph) and the host time inside the calls
+    eager = None
+    if not args.no_eager:
+        warm(step_fn, 3, stream, torch)
+        dev_ms, host_ms = time_eager(step_fn, EAGER_STEPS, stream, torch)
+        dev_ms = reduce_over_ranks(dev_ms, 0, 0, 0, device, world)[0]
+        assert sg.device_error(device) == 0, "a kernel reported a device-side error"
+        e_ach = call_bytes / (dev_ms / (EAGER_STEPS * calls_per_step) * 1e-3) / 1e9
+        eager = {"ms_per_step": dev_ms / EAGER_STEPS, "steps": EAGER_STEPS,
+                 "value": all_bytes * EAGER_STEPS / (dev_ms * 1e-3) / 1e9, "unit": "GB/s",
+                 "achieved": e_ach, "frac": e_ach / peak,
+                 "host_us_per_call": host_ms * 1e3 / (EAGER_STEPS * calls_per_step),
+                 "note": "back-to-back calls through the C ABI without a CUDA graph; host_us_per_call is the "
+                         "host time from entry to return of one call (validation, plan, tensor maps, launch)"}
+
     # ---- end to end: pinned host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        phx, phy = hx.pin_memory(), hy.pin_memory()
-        phws = [w.pin_memory() for w in hws]
-        phmeta = [m.pin_memory() for m in hmeta]
+        phx, phy = r.hx.pin_memory(), r.hy.pin_memory()
+        phws = [w.pin_memory() for w in r.hws]
+        phmeta = [m.pin_memory() for m in r.hmeta]
         out_host = torch.empty_like(phy).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in [phx, phy, *phws, *phmeta])
         d2h = out_host.numel() * out_host.element_size()
@@ -439,14 +591,14 @@ def bench_ours(args, rank, world, device):
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(E):
-                x.copy_(phx, non_blocking=True)
-                y.copy_(phy, non_blocking=True)
-                for w, pw in zip(ws, phws):
+                r.x.copy_(phx, non_blocking=True)
+                r.y.copy_(phy, non_blocking=True)
+                for w, pw in zip(r.ws, phws):
                     w.copy_(pw, non_blocking=True)
-                for m, pm in zip(meta, phmeta):
+                for m, pm in zip(r.meta, phmeta):
                     m.copy_(pm, non_blocking=True)
                 step_fn(stream.cuda_stream)
-                out_host.copy_(y, non_blocking=True)
+                out_host.copy_(r.y, non_blocking=True)
             e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -458,13 +610,10 @@ def bench_ours(args, rank, world, device):
     # ---- the same step as ONE fused multi-slice launch (several slices only)
     fused = None
     if ncalls > 1 and not args.no_fused and not fused_step:
-        run_multi = make_multi_call(p, (x, ws, y, meta))
-        fv, fl = sg.plan_multi_slice(x, ws, y, *meta, p.batches, p.max_seq_len,
+        run_multi = r.multi_call()
+        fv, fl = sg.plan_multi_slice(r.x, r.ws, r.y, *r.meta, p.batches, p.max_seq_len,
                                      [c.slice_offset for c in p.calls], p.add_inputs)
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                run_multi(stream.cuda_stream)
-        torch.cuda.synchronize()
+        warm(run_multi, args.warmup, stream, torch)
         if world > 1:
             torch.distributed.barrier()
         fms = time_graph_region(run_multi, K, stream, torch)
@@ -477,46 +626,64 @@ def bench_ours(args, rank, world, device):
                  "achieved": f_ach, "frac": f_ach / peak, "bytes_per_launch": step_bytes / max(fl, 1),
                  "note": "all slices of a step in one call; same bytes as the separate calls"}
 
+    # ---- the other workloads, each graph-timed on its own inputs (rank 0's figures)
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        main_call_us = avg_launch_ms * 1e3
+        configs[args.workload] = {
+            "workload": WORKLOAD_TEXT[args.workload], "variant": r.variant, "calls_per_step": calls_per_step,
+            "us_per_call": main_call_us, "gb_s": achieved, "frac": achieved / peak,
+            "tokens_per_s": p.total_tokens * K / (total_ms * 1e-3), "tflops": step_flops * K / (total_ms * 1e-3) / 1e12,
+            "bytes_per_call": call_bytes, "steps": K, "traffic": recorded_traffic(args.workload, r.kernel_family),
+            "note": "the headline figures above"}
+        for name in CONFIG_WORKLOADS:
+            if name == args.workload:
+                continue
+            configs[name] = secondary_entry(name, args.seed + rank, max(SECONDARY_STEPS, K), args.warmup, device,
+                                            peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(p, budget_s=args.cpu_seconds)
 
+    trafrec = recorded_traffic_split(args.workload, r.kernel_family)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": p.w_dt, "accumulate": "f32",
         "data": "synthetic (seeded numpy; inputs resident in HBM)",
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
-                   "batches": p.batches, "tokens_per_rank": p.total_tokens,
-                   "active_tokens_per_rank": step_rows // max(ncalls, 1), "rank": p.rank,
-                   "slices": ncalls, "slice_size": p.calls[0].slice_size,
-                   "adapters": int(p.calls[0].w.shape[0]), "add_inputs": bool(p.add_inputs),
-                   "x_dtype": p.x_dt, "w_dtype": p.w_dt, "out_dtype": p.out_dt,
-                   "parallelism": f"replicas x{world} (independent batches, no collective)",
-                   "l2": "no flush: every step streams the whole output, larger than L2",
-                   "variant": variant_name, "seed": args.seed,
-                   "step": ("all slices in one sgmv_expand_multi_slice call" if fused_step else
-                            f"{ncalls} separate call(s)"),
-                   "timing": f"CUDA graphs of <= {STEPS_PER_GRAPH} steps; events around the timed region"},
+        "config": workload_config(p, args.workload, world, fused_step),
+        "variant": r.variant,
+        "timing": f"CUDA graphs of <= {STEPS_PER_GRAPH} steps; events around the timed region",
         "tokens_per_s": all_tokens * K / (total_ms * 1e-3),
         "tokens_per_s_note": "batch tokens per second, all ranks (a step updates every slice of every token)",
         "tflops": all_flops * K / (total_ms * 1e-3) / 1e12,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload, kernel_family),
+                     "frac": achieved / peak, "traffic": trafrec["traffic"] if trafrec else None,
+                     "dram_read": trafrec["read"] if trafrec else None,
+                     "dram_write": trafrec["write"] if trafrec else None,
+                     "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the current "
+                                     "kernel source; reads are complete, writes still dirty in L2 when the launch "
+                                     "ends are not counted, so dram_read is the figure to hold against the "
+                                     "algorithmic reads",
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6650 GB/s",
                      "kernel": f"{ {'bgmv': 'bgmv_expand_slice', 'shrink': 'sgmv_shrink'}.get(p.op, 'sgmv_expand_slice') } "
-                               f"({variant_name}{', %d H splits + reduction' % shrink_splits if shrink_splits > 1 else ''})",
+                               f"({r.variant}{', %d H splits + reduction' % r.shrink_splits if r.shrink_splits > 1 else ''})",
                      "launch_ms_avg": avg_launch_ms, "bytes_per_launch": call_bytes,
                      "launches_timed": K * calls_per_step,
                      "launch_ms_note": "timed region / calls (back-to-back calls, gaps included; a split shrink "
                                        "call is its main kernel plus the reduction)"},
         "gpu_launches": K * launches_per_step,
         "clocks": clocks,
+        "l2_flushed": flushed,
+        "eager": eager,
         "fused_multi_slice": fused,
+        "configs": configs,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "when": datetime.datetime.utcnow().isoformat() + "Z",
+        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }
     return line
 
@@ -603,7 +770,7 @@ def bench_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": tot_t / max(args.steps, 1) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "seed": args.seed},
+            "config": workload_config(p, args.workload, world),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
                              "sample": sample_txt},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -627,6 +794,9 @@ def main():
     ap.add_argument("--step", choices=["calls", "fused"], default="calls",
                     help="time each step as separate slice calls (default) or as one multi-slice call")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-configs", action="store_true", help="skip the figures of the other workloads")
+    ap.add_argument("--no-flush", action="store_true", help="skip the L2-flushed median timing")
+    ap.add_argument("--no-eager", action="store_true", help="skip the eager (no graph) timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

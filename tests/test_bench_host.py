@@ -73,10 +73,11 @@ def _fake_root(tmp_path, source_text):
 def test_recorded_traffic_only_for_the_source_it_was_taken_on(tmp_path, monkeypatch):
     root = _fake_root(tmp_path, "v1 ")
     monkeypatch.setattr(bench, "ROOT", str(root))
-    rec = {"qkv_prefill": {"tc": {"dram_bytes_per_launch": 123.0,
+    rec = {"qkv_prefill": {"tc": {"dram_read_bytes_per_launch": 100.0, "dram_write_bytes_per_launch": 23.0,
                                   "kernel_source_hash": bench.kernel_source_hash("tc")}}}
     (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert bench.recorded_traffic("qkv_prefill", "tc") == 123.0
+    assert bench.recorded_traffic_split("qkv_prefill", "tc") == {"traffic": 123.0, "read": 100.0, "write": 23.0}
     assert bench.recorded_traffic("qkv_prefill", "decode") is None      # no record for that kernel
     assert bench.recorded_traffic("decode_mix", "tc") is None           # nor for that workload
     # a change to a file outside the family keeps the record
@@ -90,7 +91,7 @@ def test_recorded_traffic_only_for_the_source_it_was_taken_on(tmp_path, monkeypa
 def test_comment_and_layout_edits_keep_the_record(tmp_path, monkeypatch):
     root = _fake_root(tmp_path, "int v1; ")
     monkeypatch.setattr(bench, "ROOT", str(root))
-    rec = {"qkv_prefill": {"tc": {"dram_bytes_per_launch": 5.0,
+    rec = {"qkv_prefill": {"tc": {"dram_read_bytes_per_launch": 4.0, "dram_write_bytes_per_launch": 1.0,
                                   "kernel_source_hash": bench.kernel_source_hash("tc")}}}
     (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
     f = root / "segmented_gather_gemm_expand_b200" / "csrc" / "tc_kernel.cuh"
@@ -116,7 +117,7 @@ def test_committed_traffic_records_are_well_formed():
         assert workload in gen.WORKLOADS, workload
         for family, e in kernels.items():
             assert family in bench.KERNEL_SOURCES, family
-            assert e["dram_bytes_per_launch"] > 0
+            assert e["dram_read_bytes_per_launch"] > 0 and e["dram_write_bytes_per_launch"] >= 0
             assert len(e["kernel_source_hash"]) == 16
             assert os.path.exists(os.path.join(bench.ROOT, e["source"].split(" ")[0]))
 
@@ -141,6 +142,10 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["name"] == "qkv_prefill"
+    # the same workload description our arm prints, so the two lines compare like for like
+    import numpy as np  # noqa: F401
+    p = gen.WORKLOADS["qkv_prefill"](seed=0)
+    assert d["config"] == json.loads(json.dumps(bench.workload_config(p, "qkv_prefill", 1)))
 
 
 def test_reference_arm_under_two_ranks_prints_once():

@@ -354,7 +354,7 @@ def test_more_pieces_per_cta_than_ring_slots(case, variant):
     short = rng.random(B) < MANY_PIECES[case]["short_share"]
     lengths = np.where(short, rng.integers(1, 128, B), 128)
     idx = rng.integers(-1, 8, B)
-    N = 1280                           # 10 n-tiles of 128 columns, 5 of 256
+    N = 1536                           # 12 n-tiles of 128 columns, 6 of 256
     p = gen.custom(seed=79, lengths=lengths.tolist(), K=16, N=N, H=N + 256, offset=128, num_adapters=8,
                    idx=idx.tolist())
     dp = DeviceProblem(p)

@@ -33,7 +33,7 @@ constexpr int BM = 128;               // rows per block (TMEM lanes)
 constexpr int CH = 64;                // H columns per chunk: 128-byte rows
 constexpr int THREADS = 192;
 constexpr int NUM_ACC = 2;
-constexpr int SEG_CAP = 1024;
+constexpr int SEG_CAP = 16384;        // most segments a launch takes (the shared-memory table decides below that)
 constexpr int NUM_XMAPS = 5;          // x boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_RANK = 128;
 constexpr int SMEM_LIMIT = 232448 - 1024;   // dynamic shared memory a CTA may opt in to on sm_100
@@ -353,14 +353,13 @@ inline bool supports(const Problem& p) {
     if ((reinterpret_cast<uintptr_t>(p.x) & 15) || (reinterpret_cast<uintptr_t>(p.w) & 15) ||
         (reinterpret_cast<uintptr_t>(p.out) & 15))
         return false;
-    if (p.batches > SEG_CAP) return false;
     if (p.out_rows >= (int64_t(1) << 31) || p.x_rows >= (int64_t(1) << 31) || p.lora_num >= (int64_t(1) << 31))
         return false;
     return true;
 }
 
 inline bool make_plan(const Problem& p, int sm_count, int splits, tc::EncodeTiledFn enc, Plan* out) {
-    if (!supports(p) || !enc) return false;
+    if (!supports(p) || !enc || p.batches > SEG_CAP) return false;
     Geo& g = out->geo;
     g.R = (int32_t)p.N;
     g.nchunks = (int32_t)((p.K + CH - 1) / CH);

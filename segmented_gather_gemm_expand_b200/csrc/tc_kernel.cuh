@@ -1,16 +1,22 @@
 // Tensor-core SGMV expand-slice for sm_100a: tcgen05 MMA with the accumulator
 // in tensor memory, TMA staging of B, x and the output slice.
 //
-// One persistent CTA per SM, 352 threads in warp roles.  BN, the n-tile width,
+// One persistent CTA per SM, 384 threads in warp roles.  BN, the n-tile width,
 // is 128 or 256 columns (a template parameter); TMEM holds 512 / BN accumulators.
 //
-//   warp 0    producer   TMA: x for each 128-row block of a segment and B[a]'s
-//                        BN-row n-tile (K in 64/32/16/8-column boxes with the
-//                        matching swizzle) for each piece.
-//   warp 2    loader     allocates each piece's rows in shared-memory rings (one
-//                        ring of 128-byte rows per 128-byte column chunk, in
-//                        piece order, freed as the epilogue's stores drain) and,
-//                        in add mode, TMA-loads the old output there: whole
+//   warp 11   scheduler  builds the segment table (the guards of sgmv.h
+//                        applied), generates this CTA's pieces (tc_sched.cuh)
+//                        and publishes them, in order, as records in a queue
+//                        in shared memory: block, columns, ring position,
+//                        x-block reuse, TMEM copy layout.  The other roles only
+//                        read records.
+//   warp 0    producer   TMA: x for each new 128-row block and B[a]'s BN-row
+//                        n-tile (K in 64/32/16/8-column boxes with the matching
+//                        swizzle) for each piece.
+//   warp 2    loader     in add mode, TMA-loads each piece's old output into
+//                        its rows of the shared-memory rings (one ring of
+//                        128-byte rows per 128-byte column chunk, in piece
+//                        order, freed as the epilogue's stores drain): whole
 //                        8-row groups as 2-D boxes of 8..128 rows (128-byte
 //                        swizzle), clipped at the slice's last column.
 //   warp 1    MMA        rounds x to the weights' dtype into the MMA operand
@@ -30,16 +36,10 @@
 //                        registers, so nothing outside the segment's rows is
 //                        written.
 //
-// Work is expanded on the device.  A piece is (segment, 128-row block of the
-// segment, n-tile); pieces are ordered with the n-tile fastest.  Every CTA
-// builds the table of segments in shared memory (the guards of sgmv.h
-// applied) and then, identically in every CTA, either deals the pieces
-// round-robin (when full and partial blocks are mixed) or gives each CTA the
-// pieces that start in its equal share of the total weight (a piece weighs its
-// 8-row groups, at least a floor, plus its B tile), keeping an x block across
-// its n-tiles.
-// Every wait on an mbarrier is bounded; a wait that gives up sets the device
-// error word and makes the CTA leave its loops.
+// A piece is (segment, 128-row block of the segment, columns of one n-tile or
+// of half of one); how pieces are handed out to CTAs is described in
+// tc_sched.cuh.  Every wait on an mbarrier is bounded; a wait that gives up
+// sets the device error word and makes the CTA leave its loops.
 #pragma once
 
 #include <cuda.h>
@@ -49,35 +49,38 @@
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
+#include "tc_sched.cuh"
 
 namespace sgmv {
 namespace tc {
 
-constexpr int BM = 128;               // rows per MMA tile (TMEM lanes)
+using sched::SegEntry;
+using sched::SliceTable;
+using sched::Piece;
+
+constexpr int BM = sched::BM;         // rows per MMA tile (TMEM lanes)
 constexpr int BM_LOG = 7;
 static_assert((1 << BM_LOG) == BM, "BM is a power of two");
-constexpr int TMEM_COLS = 512;       // every accumulator of a CTA: all of TMEM
-constexpr int GROUP = 8;              // rows per work unit
-constexpr int GROUPS_PER_BLOCK = BM / GROUP;
-constexpr int THREADS = 352;
+constexpr int TMEM_COLS = 512;        // every accumulator of a CTA: all of TMEM
+constexpr int GROUP = sched::GROUP;   // rows per work unit
+constexpr int THREADS = 384;
 constexpr int EPI_WARP0 = 3;          // first epilogue warp
 constexpr int EPI_GROUPS = 2;         // epilogue warp groups, taking pieces in turn
 constexpr int EPI_WARPS = 4 * EPI_GROUPS;
-constexpr int SEG_CAP = 1024;         // segments held in shared memory
+constexpr int SCHED_WARP = 11;
+constexpr int SEG_CAP = 16384;        // most segments a launch takes (the shared-memory table decides below that)
+constexpr int WARP_TABLE_MAX = 32;    // segment tables up to this size are built by the scheduler warp alone
 constexpr int MAX_KP = 128;           // largest padded rank
 constexpr int NUM_YMAPS = 5;          // output boxes of 8, 16, 32, 64, 128 rows
 constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
-constexpr int MAX_SLICES = 4;         // slices of one output updated by one launch
+constexpr int MAX_SLICES = sched::MAX_SLICES;   // slices of one output updated by one launch
 constexpr int RING_PIECES = 32;       // pieces that may hold ring space at once
-// an accumulator slot and a ring barrier slot always serve the same epilogue group
-static_assert(RING_PIECES % EPI_GROUPS == 0, "slot ownership");
-
-struct SegEntry {
-    int32_t row0;
-    int32_t rows;
-    int32_t adapter;
-    int32_t prefix;     // weight of all pieces of earlier segments
-};
+constexpr int QS = 64;                // piece records in the queue
+// an accumulator slot, a ring barrier slot and a queue slot always serve the same epilogue group
+static_assert(RING_PIECES % EPI_GROUPS == 0 && QS % EPI_GROUPS == 0, "slot ownership");
+constexpr int32_t MODE_AUTO = -1;     // Geometry::mode: decided on the device from the segment table
+// record slot readers: producer, loader, MMA warp, and the four warps of the piece's epilogue group
+constexpr uint32_t QUEUE_READERS = 3 + 4;
 
 // Geometry fixed per launch (host computes; kernel parameter).
 struct Geometry {
@@ -88,8 +91,10 @@ struct Geometry {
     int32_t n_tiles;    // n-tiles of all slices together
     int32_t ring_rows, stages_w, stages_xo, stages_xr;
     int32_t w_is_bf16;
-    int32_t wmin, wfix; // scheduling weight of a piece: max(its 8-row groups, wmin) + wfix
-    int32_t rr;         // 1: the kernel may hand out pieces round-robin (see the segment table)
+    int32_t wmin, wfix; // contiguous mode: weight of a piece = max(its 8-row groups, wmin) + wfix
+    int32_t mode;       // sched::MODE_CONTIG, or MODE_AUTO: the kernel picks (choose_mode)
+    int32_t spread;     // MODE_AUTO's choice for batches of mostly full blocks: MODE_RR or MODE_BALANCED
+    int32_t halves;     // balanced mode: 2 = the tail is dealt in column halves
     int32_t bn;         // columns per n-tile: 128 or 256 (the kernel's BN)
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
     // (rows of 2*kb bytes, swizzled by the row width) at w_blk_off in a stage
@@ -103,7 +108,7 @@ struct Geometry {
     uint32_t b_off[MAX_KP / 16];
 
     // shared memory offsets (bytes, from the 1024-aligned base)
-    int32_t off_y, off_w, off_xo, off_xr, off_seg, off_ends, off_bar;
+    int32_t off_y, off_w, off_xo, off_xr, off_seg, off_inv, off_ends, off_q, off_bar;
     int32_t w_bytes, xo_bytes, xr_bytes;
 };
 
@@ -115,11 +120,9 @@ struct WMaps {
     CUtensorMap m[MAX_SLICES][MAX_WBLK];
 };
 
-
-
-// The slices of one launch: slice s covers output columns [off[s], off[s] + N[s])
-// with its own B; its n-tiles are numbers [tile0[s], tile0[s + 1]) of a piece's
-// row block.
+// The slices of one launch (kernel parameter); copied into shared memory as a
+// SliceTable, since reading it from the parameter space through a pointer
+// with a data-dependent index costs a slow generic load on every piece.
 struct Slices {
     int32_t count;
     int32_t tile0[MAX_SLICES + 1];
@@ -127,205 +130,51 @@ struct Slices {
     int64_t N[MAX_SLICES];
 };
 
-// The slice table as the kernel reads it, copied into shared memory at the
-// start: reading it from the parameter space through a pointer with a
-// data-dependent index costs a slow generic load on every piece.
-struct SliceTable {
-    int32_t tile0[MAX_SLICES + 1];
-    int32_t off[MAX_SLICES];
-    int32_t N[MAX_SLICES];
-};
+// ---------------------------------------------------------------- piece records
 
-// ---------------------------------------------------------------- scheduler
+enum : int32_t { REC_NEW_X = 1, REC_LAST_X = 2, REC_END = 4, REC_NEW_W = 8, REC_LAST_W = 16 };
 
-struct Piece {
+// One piece as the roles read it from the queue.
+struct PieceRec {
     int32_t adapter;
     int32_t blk_row0;     // row (of out and x) where the 128-row block starts
     int32_t rows;         // rows of the block (1 .. 128)
     int32_t n0;           // first column within the slice
     int32_t col0;         // first output column of the piece
-    int32_t ncols;        // columns of the piece (1 .. the n-tile width)
+    int32_t ncols;        // columns of the piece
     int32_t slice;
     int32_t rep_log;      // log2 of the copies of the piece's rows in TMEM (1, 2 or 4 copies,
                           // one per 128/copies lanes)
     int32_t shift;        // lane of the piece's first row within each copy (0, 32, 64 or 96)
-    int32_t t;            // index of the piece among this CTA's pieces
-    bool new_x;           // first piece of this x block in this CTA
-    bool last_x;          // last piece of this x block in this CTA
+    int32_t pos;          // first ring row of the piece
+    int32_t head_end;     // ring rows handed out up to and including this piece
+    int32_t flags;        // REC_NEW_X / REC_LAST_X: first / last piece of its x block in this CTA;
+                          // REC_NEW_W / REC_LAST_W: the same for its B tile (adapter, slice, first column)
 };
 
 // log2 of the lanes between repeats of a block's rows in the staged x operand:
 // the rows rounded up to 32, 64 or 128.
-__device__ __forceinline__ int32_t x_period_log(int32_t rows) { return rows <= 32 ? 5 : rows <= 64 ? 6 : BM_LOG; }
+__host__ __device__ __forceinline__ int32_t x_period_log(int32_t rows) { return rows <= 32 ? 5 : rows <= 64 ? 6 : BM_LOG; }
 
-// Walks the CTA's pieces in one of two ways:
-//   - contiguous: the pieces whose start weight lies in [w0, w_end) (seek);
-//   - round-robin: pieces c, c + stride, c + 2*stride, ... of the sequence of all
-//     pieces (seek_rr), so that every CTA gets the same mix of long and short
-//     pieces and, at any moment, the CTAs together cover whole output rows.
-// Every role runs an identical copy, so all roles see the same sequence.
-struct Walker {
-    const SegEntry* segs;
-    const SliceTable* st;   // shared memory
-    int32_t nseg, n_tiles, wmin, wfix;
-    int32_t bn;           // columns per n-tile
-    int32_t cc_log;       // log2 of the columns per 128-byte output chunk
-    int32_t i, rb, j;     // segment, row block, n-tile
-    int32_t t;            // pieces handed out so far
-    int32_t G, nblk, gcw; // groups and blocks of segment i; weight of a piece of block rb
-    int32_t cur, w_end;   // start weight of the next piece; end of the range
-    int32_t stride;       // round-robin stride (0: contiguous)
-    bool first;
+// Place a piece of rows8 rows in a ring of R rows: returns the ring row where it
+// starts and advances `head` (rows handed out so far, including skipped ones).
+// A piece never wraps: if it does not fit before the ring's end it starts at 0.
+__device__ __forceinline__ int32_t ring_place(int32_t& head, int32_t rows8, int32_t R) {
+    int32_t pos = head % R;
+    if (pos + rows8 > R) {
+        head += R - pos;
+        pos = 0;
+    }
+    head += rows8;
+    return pos;
+}
 
-    __device__ void load_segment_geometry() {
-        G = (segs[i].rows + GROUP - 1) / GROUP;
-        nblk = (G + GROUPS_PER_BLOCK - 1) / GROUPS_PER_BLOCK;
-    }
-    __device__ void set_block() { gcw = max(min(GROUPS_PER_BLOCK, G - rb * GROUPS_PER_BLOCK), wmin) + wfix; }
-    __device__ void skip_empty() {
-        while (i < nseg && segs[i].rows == 0) ++i;
-        if (i < nseg) {
-            load_segment_geometry();
-            cur = segs[i].prefix;
-        }
-    }
-
-    __device__ void seek(int32_t w0, int32_t w1) {
-        w_end = w1;
-        stride = 0;
-        first = true;
-        t = 0;
-        i = nseg;
-        rb = j = 0;
-        cur = w1;
-        if (w0 >= w1) return;
-        int lo = 0, hi = nseg - 1;   // last segment whose prefix <= w0
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) / 2;
-            if (segs[mid].prefix <= w0) lo = mid;
-            else hi = mid - 1;
-        }
-        i = lo;
-        skip_empty();
-        if (i >= nseg) return;
-        const int32_t local = w0 - segs[i].prefix;
-        const int32_t bw = (max(GROUPS_PER_BLOCK, wmin) + wfix) * n_tiles;   // weight of a full row block
-        rb = min(local / bw, nblk - 1);
-        set_block();
-        const int32_t rem = local - rb * bw;
-        j = (rem + gcw - 1) / gcw;                              // first piece starting at or after w0
-        if (j >= n_tiles) {
-            j = 0;
-            if (++rb == nblk) {
-                rb = 0;
-                ++i;
-                skip_empty();
-                if (i >= nseg) return;
-                cur = segs[i].prefix;
-                set_block();
-                return;
-            }
-            set_block();
-        }
-        cur = segs[i].prefix + rb * bw + j * gcw;
-    }
-
-    // Round-robin: the segment table's prefixes count pieces.  Moves to piece
-    // `local` of segment i (or of a later segment), skipping empty ones.
-    __device__ void advance_rr(int32_t local) {
-        while (i < nseg && local >= nblk * n_tiles) {
-            local -= nblk * n_tiles;
-            ++i;
-            while (i < nseg && segs[i].rows == 0) ++i;
-            if (i < nseg) load_segment_geometry();
-        }
-        rb = local / n_tiles;
-        j = local - rb * n_tiles;
-    }
-
-    __device__ void seek_rr(int32_t c, int32_t step) {
-        stride = step;
-        first = true;
-        t = 0;
-        i = nseg;
-        rb = j = 0;
-        if (nseg == 0) return;
-        int lo = 0, hi = nseg - 1;   // last segment whose prefix <= c
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) / 2;
-            if (segs[mid].prefix <= c) lo = mid;
-            else hi = mid - 1;
-        }
-        i = lo;
-        while (i < nseg && segs[i].rows == 0) ++i;
-        if (i >= nseg) return;
-        load_segment_geometry();
-        advance_rr(c - segs[i].prefix);
-    }
-
-    __device__ bool next_rr(Piece& p) {
-        if (i >= nseg) return false;
-        const int32_t pi = i, prb = rb;
-        fill(p);
-        p.new_x = first || i != last_i || rb != last_rb;
-        first = false;
-        last_i = i;
-        last_rb = rb;
-        advance_rr(rb * n_tiles + j + stride);
-        p.last_x = i >= nseg || i != pi || rb != prb;
-        return true;
-    }
-    int32_t last_i, last_rb;
-
-    // The piece at (i, rb, j), and the quadrant turn of the t-th piece.
-    __device__ void fill(Piece& p) {
-        const SegEntry s = segs[i];
-        p.adapter = s.adapter;
-        p.blk_row0 = s.row0 + rb * BM;
-        p.rows = min(BM, s.rows - rb * BM);
-        int32_t sl = 0;
-        while (j >= st->tile0[sl + 1]) ++sl;
-        p.slice = sl;
-        p.n0 = (j - st->tile0[sl]) * bn;
-        p.col0 = st->off[sl] + p.n0;
-        p.ncols = min(bn, st->N[sl] - p.n0);
-        // A short piece (rows in 1 or 2 quadrants) is computed in every span
-        // of 32 or 64 lanes: the x block is staged with its rows repeated
-        // (x_period), so each TMEM quadrant holds a copy of the sums, and the
-        // epilogue warps of the copies split the piece's column chunks.  Where
-        // the piece has fewer chunks than copies, its rows instead take turns
-        // in the lanes of a wider span (the pieces of one epilogue group,
-        // every EPI_GROUPS-th, cycle through them).
-        // (all powers of two: shifts and masks only, this runs for every piece in every role)
-        const int32_t span_log = x_period_log(p.rows);
-        const int32_t nch = (p.ncols + (1 << cc_log) - 1) >> cc_log;
-        const int32_t maxrep_log = BM_LOG - span_log;
-        p.rep_log = min(maxrep_log, nch >= 4 ? 2 : nch >= 2 ? 1 : 0);
-        const int32_t turns_mask = (1 << (maxrep_log - p.rep_log)) - 1;
-        p.shift = ((t / EPI_GROUPS) & turns_mask) << span_log;
-        p.t = t++;
-    }
-
-    __device__ bool next(Piece& p) {
-        if (stride) return next_rr(p);
-        if (i >= nseg || cur >= w_end) return false;
-        fill(p);
-        p.new_x = first || j == 0;
-        first = false;
-        cur += gcw;
-        if (++j == n_tiles) {
-            j = 0;
-            if (++rb == nblk) {
-                rb = 0;
-                ++i;
-                skip_empty();
-            }
-            if (i < nseg) set_block();
-        }
-        p.last_x = j == 0 || i >= nseg || cur >= w_end;
-        return true;
-    }
-};
+// Index k of the largest output box (8 << k rows, k <= max_level) that fits in
+// `rows` (a positive multiple of 8).
+__device__ __forceinline__ int box_level(int rows, int max_level) {
+    const int k = 31 - __clz(rows / GROUP);
+    return k < max_level ? k : max_level;
+}
 
 // Exclusive block-wide scan of units_of(segs[b]) into segs[b].prefix; returns
 // the total.  Called by all THREADS threads; ends synchronised.
@@ -357,24 +206,55 @@ __device__ int32_t scan_segments(SegEntry* segs, int32_t nseg, int32_t* warp_sum
     return running;
 }
 
-// Index k of the largest output box (8 << k rows, k <= max_level) that fits in
-// `rows` (a positive multiple of 8).
-__device__ __forceinline__ int box_level(int rows, int max_level) {
-    const int k = 31 - __clz(rows / GROUP);
-    return k < max_level ? k : max_level;
+// Segment units of the scan: full-block pieces (balanced), all pieces (round-robin) or weight (contiguous).
+__device__ __forceinline__ int32_t seg_units(const Geometry& geo, int32_t mode, int32_t rows) {
+    if (mode == sched::MODE_BALANCED) return sched::full_pieces(rows, geo.n_tiles);
+    if (mode == sched::MODE_RR || mode == sched::MODE_COLS) return sched::all_pieces(rows, geo.n_tiles);
+    return sched::contig_weight(rows, geo.n_tiles, geo.wmin, geo.wfix);
 }
 
-// Place a piece of rows8 rows in a ring of R rows: returns the ring row where it
-// starts and advances `head` (rows handed out so far, including skipped ones).
-// A piece never wraps: if it does not fit before the ring's end it starts at 0.
-__device__ __forceinline__ int32_t ring_place(int32_t& head, int32_t rows8, int32_t R) {
-    int32_t pos = head % R;
-    if (pos + rows8 > R) {
-        head += R - pos;
-        pos = 0;
+// How this launch hands out pieces (the same in every CTA).  A batch whose row
+// blocks are mostly partial (short segments: decode-like mixes) takes
+// contiguous ranges, which keep each x block and walk one adapter's B tiles in
+// order; others take geo.spread (their pieces are dealt across the CTAs).
+__device__ __forceinline__ int32_t choose_mode(const Geometry& geo, int32_t partial_blocks, int32_t blocks) {
+    if (geo.mode != MODE_AUTO) return geo.mode;
+    return 2 * partial_blocks > blocks ? (int32_t)sched::MODE_CONTIG : geo.spread;
+}
+
+// The sorted tail of the balanced mode, built by the scheduler warp: bucket
+// counts and the segments of each bucket in index order (ballots over chunks
+// of 32 segments, so every CTA builds the same table).
+__device__ void build_tail(const SegEntry* segs, int32_t nseg, int32_t total, int32_t n_tiles, int32_t halves,
+                           sched::Tail* tl, int32_t* inv) {
+    const int lane = threadIdx.x % 32;
+    const uint32_t lt = (1u << lane) - 1u;
+    int32_t cnt[sched::NUM_BUCKETS + 1];
+#pragma unroll
+    for (int r = 0; r <= sched::NUM_BUCKETS; ++r) cnt[r] = 0;
+    for (int32_t base = 0; base < nseg; base += 32) {
+        const int32_t s = base + lane;
+        const int32_t r = s < nseg ? sched::partial_bucket(segs[s].rows) : 0;
+#pragma unroll
+        for (int q = 1; q <= sched::NUM_BUCKETS; ++q) cnt[q] += __popc(__ballot_sync(0xffffffffu, r == q));
     }
-    head += rows8;
-    return pos;
+    sched::Tail t;
+    sched::tail_layout(t, cnt, total, (int32_t)gridDim.x, n_tiles, halves);
+    int32_t fill[sched::NUM_BUCKETS + 1];
+#pragma unroll
+    for (int q = 0; q <= sched::NUM_BUCKETS; ++q) fill[q] = q ? t.seg0[q] : 0;
+    for (int32_t base = 0; base < nseg; base += 32) {
+        const int32_t s = base + lane;
+        const int32_t r = s < nseg ? sched::partial_bucket(segs[s].rows) : 0;
+#pragma unroll
+        for (int q = 1; q <= sched::NUM_BUCKETS; ++q) {
+            const uint32_t m = __ballot_sync(0xffffffffu, r == q);
+            if (r == q) inv[fill[q] + __popc(m & lt)] = s;
+            fill[q] += __popc(m);
+        }
+    }
+    if (lane == 0) *tl = t;
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -393,16 +273,18 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
 
     __shared__ int s_abort;
     __shared__ uint32_t s_tmem_base;
-    __shared__ int32_t s_total_units;
     __shared__ int32_t s_warp_sums[THREADS / 32];
-    __shared__ int32_t s_partial_pieces;
     __shared__ SliceTable s_sl;
+    __shared__ sched::Tail s_tail;
+    __shared__ int32_t s_blocks, s_partial;   // row blocks and partial ones (long tables)
 
     const int tid = threadIdx.x;
     const int warp = tid / 32;
     const int lane = tid % 32;
 
     SegEntry* segs = reinterpret_cast<SegEntry*>(smem + geo.off_seg);
+    int32_t* inv = reinterpret_cast<int32_t*>(smem + geo.off_inv);
+    PieceRec* recs = reinterpret_cast<PieceRec*>(smem + geo.off_q);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + geo.off_bar);
     const int SW = geo.stages_w, SXO = geo.stages_xo, SXR = geo.stages_xr;
     const int32_t R = geo.ring_rows;
@@ -416,10 +298,13 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     uint64_t* acc_empty = acc_full + NUM_ACC;
     uint64_t* y_full = acc_empty + NUM_ACC;     // piece's ring rows ready (loaded, in add mode)
     uint64_t* y_free = y_full + RING_PIECES;     // piece's ring rows no longer read by any store
+    uint64_t* q_full = y_free + RING_PIECES;     // queue slot holds a record
+    uint64_t* q_empty = q_full + QS;             // queue slot read by every reader
 
     if (tid == 0) {
         s_abort = 0;
-        s_partial_pieces = 0;
+        s_blocks = 0;
+        s_partial = 0;
         for (int i = 0; i <= MAX_SLICES; ++i) s_sl.tile0[i] = sl.tile0[i];
         for (int i = 0; i < MAX_SLICES; ++i) {
             s_sl.off[i] = (int32_t)sl.off[i];
@@ -428,13 +313,17 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     }
     {
         // The barriers lie back to back from w_full; every thread initialises a
-        // few.  acc_empty and y_free count the four warps of an epilogue group.
-        const int n_bars = (int)(y_free + RING_PIECES - bars);
+        // few.  acc_empty and y_free count the four warps of an epilogue group,
+        // q_empty every reader of a record.
+        const int n_bars = (int)(q_empty + QS - bars);
         const int acc_empty0 = (int)(acc_empty - bars), y_free0 = (int)(y_free - bars);
+        const int q_empty0 = (int)(q_empty - bars);
         bool did = false;
         for (int b = tid; b < n_bars; b += THREADS) {
-            const bool four = (b >= acc_empty0 && b < acc_empty0 + NUM_ACC) || b >= y_free0;
-            mbar_init(smem_u32(&bars[b]), four ? 4u : 1u);
+            uint32_t count = 1;
+            if ((b >= acc_empty0 && b < acc_empty0 + NUM_ACC) || (b >= y_free0 && b < y_free0 + RING_PIECES)) count = 4;
+            if (b >= q_empty0) count = QUEUE_READERS;
+            mbar_init(smem_u32(&bars[b]), count);
             did = true;
         }
         if (did) fence_barrier_init();
@@ -475,86 +364,159 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             prefetch_l2(static_cast<const char*>(m->ptr) + b * m->stride * esz);
         }
     }
-
-    // Everything below may read memory written by the preceding kernel.
-    grid_dependency_wait();
-
-    // Segment table: guards of the API applied.
-    const int32_t nseg = (int32_t)p.batches;
-    for (int32_t b = tid; b < nseg; b += THREADS) {
-        const Segment s = load_segment(p, b);
-        segs[b] = SegEntry{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0};
-    }
-    __syncthreads();
-    // Pieces per segment, and how many belong to partial (< 128-row) blocks.
-    int32_t my_partial = 0;
-    for (int32_t b = tid; b < nseg; b += THREADS)
-        if (segs[b].rows % BM) my_partial += geo.n_tiles;
-    if (my_partial) atomicAdd(&s_partial_pieces, my_partial);
-    const int32_t n_tiles = geo.n_tiles;
-    const int32_t total_pieces = scan_segments(segs, nseg, s_warp_sums, [&](const SegEntry& e) {
-        return (e.rows + BM - 1) / BM * n_tiles;
-    });
-    // Round-robin when long and short pieces are mixed: equal-weight ranges of
-    // the piece sequence then split unevenly, while every CTA's round-robin
-    // share is a fair sample.  With pieces all alike, contiguous ranges are
-    // already even and keep each CTA's x block in use across its n-tiles.
-    const int32_t partial = s_partial_pieces;   // complete: scan_segments synchronises
-    const bool rr = geo.rr && partial > 0 && 2 * partial <= total_pieces;
-    int32_t running = total_pieces;
-    if (!rr) {
-        const int32_t wmin = geo.wmin, wfix = geo.wfix;
-        running = scan_segments(segs, nseg, s_warp_sums, [&](const SegEntry& e) {
-            const int32_t G = (e.rows + GROUP - 1) / GROUP;
-            if (G == 0) return 0;
-            const int32_t full = (G - 1) / GROUPS_PER_BLOCK;          // full 128-row blocks
-            const int32_t last = G - full * GROUPS_PER_BLOCK;         // groups of the last block
-            return (full * max(GROUPS_PER_BLOCK, wmin) + max(last, wmin) + (full + 1) * wfix) * n_tiles;
-        });
-    }
-    if (tid == 0) s_total_units = running;
-    grid_dependents_launch();
-
+    // barriers, the TMEM address, the slice table and the zeroed padding are
+    // visible to every role from here
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    const uint32_t tmem_base = s_tmem_base;
-    const int32_t U = s_total_units;
-    Walker walk;
-    walk.segs = segs;
-    walk.st = &s_sl;
-    walk.nseg = nseg;
-    walk.n_tiles = geo.n_tiles;
-    walk.wmin = geo.wmin;
-    walk.bn = BN;
-    walk.cc_log = OUT_BYTES == 4 ? 5 : 6;
-    walk.wfix = geo.wfix;
-    if (rr)
-        walk.seek_rr((int32_t)blockIdx.x, (int32_t)gridDim.x);
-    else
-        walk.seek((int32_t)(((int64_t)U * blockIdx.x) / gridDim.x), (int32_t)(((int64_t)U * (blockIdx.x + 1)) / gridDim.x));
+    // Everything below may read memory written by the preceding kernel.
+    grid_dependency_wait();
+    // The next kernel may be scheduled now: its CTAs take SMs as ours leave, and
+    // it waits for this grid to finish before it reads anything.
+    grid_dependents_launch();
 
+    const int32_t nseg = (int32_t)p.batches;
+    int32_t long_table_total = 0, long_table_mode = 0;   // every thread gets the scan's total and the mode
+    if (nseg > WARP_TABLE_MAX) {
+        // a long segment table: every thread loads and scans (ends synchronised)
+        int32_t my_blocks = 0, my_partial = 0;
+        for (int32_t b = tid; b < nseg; b += THREADS) {
+            const Segment s = load_segment(p, b);
+            segs[b] = SegEntry{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0};
+            my_blocks += (int32_t)((s.rows + BM - 1) / BM);
+            my_partial += (s.rows % BM) != 0;
+        }
+        if (my_blocks) atomicAdd(&s_blocks, my_blocks);
+        if (my_partial) atomicAdd(&s_partial, my_partial);
+        __syncthreads();
+        long_table_mode = choose_mode(geo, s_partial, s_blocks);
+        long_table_total = scan_segments(segs, nseg, s_warp_sums, [&](const SegEntry& e) {
+            return seg_units(geo, long_table_mode, e.rows);
+        });
+    }
+
+    const uint32_t tmem_base = s_tmem_base;
     volatile int* abort_flag = &s_abort;
     const bool w_bf16 = geo.w_is_bf16 != 0;
     constexpr int CC = 128 / OUT_BYTES;              // columns per 128-byte chunk
     constexpr int NCH = BN / CC;                     // chunks per n-tile
-
     const int32_t RING_STRIDE = R * 128;             // bytes of one chunk's ring
 
-    if (warp == 0) {
+    if (warp == SCHED_WARP) {
+        // ------------------------------------------------------------ scheduler
+        int32_t total, mode;
+        if (nseg <= WARP_TABLE_MAX) {
+            // a short table: one segment per lane, a warp scan, no block barrier
+            SegEntry e{0, 0, 0, 0};
+            if (lane < nseg) {
+                const Segment s = load_segment(p, lane);
+                e = SegEntry{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0};
+            }
+            mode = choose_mode(geo, (int32_t)__reduce_add_sync(0xffffffffu, (e.rows % BM) != 0 ? 1u : 0u),
+                               (int32_t)__reduce_add_sync(0xffffffffu, (uint32_t)((e.rows + BM - 1) / BM)));
+            const int32_t units = lane < nseg ? seg_units(geo, mode, e.rows) : 0;
+            int32_t v = units;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += t;
+            }
+            e.prefix = v - units;
+            if (lane < nseg) segs[lane] = e;
+            total = __shfl_sync(0xffffffffu, v, 31);
+            __syncwarp();
+        } else {
+            total = long_table_total;
+            mode = long_table_mode;
+        }
+        if (mode == sched::MODE_BALANCED) build_tail(segs, nseg, total, geo.n_tiles, geo.halves, &s_tail, inv);
+        if (lane == 0) {
+            sched::Gen g;
+            g.segs = segs;
+            g.st = &s_sl;
+            g.inv = inv;
+            g.tl = &s_tail;
+            g.nseg = nseg;
+            g.n_tiles = geo.n_tiles;
+            g.bn = BN;
+            g.mode = mode;
+            g.init((int32_t)blockIdx.x, (int32_t)gridDim.x, total, geo.wmin, geo.wfix);
+            constexpr int CC_LOG = OUT_BYTES == 4 ? 5 : 6;
+            Piece cur, nxt, prev;
+            bool have = g.next(cur), ok = true;
+            int32_t t = 0, head = 0, prev_seg = -1, prev_rb = -1;
+            while (have && ok) {
+                const bool have_n = g.next(nxt);
+                PieceRec r;
+                r.adapter = cur.adapter;
+                r.blk_row0 = cur.blk_row0;
+                r.rows = cur.rows;
+                r.n0 = cur.n0;
+                r.col0 = cur.col0;
+                r.ncols = cur.ncols;
+                r.slice = cur.slice;
+                r.flags = 0;
+                if (cur.seg != prev_seg || cur.rb != prev_rb) r.flags |= REC_NEW_X;
+                if (!have_n || nxt.seg != cur.seg || nxt.rb != cur.rb) r.flags |= REC_LAST_X;
+                if (t == 0 || cur.adapter != prev.adapter || cur.slice != prev.slice || cur.n0 != prev.n0)
+                    r.flags |= REC_NEW_W;
+                if (!have_n || nxt.adapter != cur.adapter || nxt.slice != cur.slice || nxt.n0 != cur.n0)
+                    r.flags |= REC_LAST_W;
+                // A short piece (rows in 1 or 2 quadrants) is computed in every span
+                // of 32 or 64 lanes: the x block is staged with its rows repeated
+                // (x_period), so each TMEM quadrant holds a copy of the sums, and the
+                // epilogue warps of the copies split the piece's column chunks.  Where
+                // the piece has fewer chunks than copies, its rows instead take turns
+                // in the lanes of a wider span (the pieces of one epilogue group,
+                // every EPI_GROUPS-th, cycle through them).
+                const int32_t span_log = x_period_log(cur.rows);
+                const int32_t nch = (cur.ncols + (1 << CC_LOG) - 1) >> CC_LOG;
+                const int32_t maxrep_log = BM_LOG - span_log;
+                r.rep_log = min(maxrep_log, nch >= 4 ? 2 : nch >= 2 ? 1 : 0);
+                const int32_t turns_mask = (1 << (maxrep_log - r.rep_log)) - 1;
+                r.shift = ((t / EPI_GROUPS) & turns_mask) << span_log;
+                r.pos = ring_place(head, (cur.rows + GROUP - 1) & ~(GROUP - 1), R);
+                r.head_end = head;
+                const int slot = t % QS;
+                if (!mbar_wait(smem_u32(&q_empty[slot]), ((t / QS) & 1) ^ 1, abort_flag, DEVERR_SCHEDULE)) {
+                    ok = false;
+                    break;
+                }
+                recs[slot] = r;
+                mbar_arrive(smem_u32(&q_full[slot]));
+                prev_seg = cur.seg;
+                prev_rb = cur.rb;
+                prev = cur;
+                cur = nxt;
+                have = have_n;
+                ++t;
+            }
+            // one end record for each epilogue group (the other roles stop at the first)
+            for (int e = 0; ok && e < EPI_GROUPS; ++e, ++t) {
+                const int slot = t % QS;
+                if (!mbar_wait(smem_u32(&q_empty[slot]), ((t / QS) & 1) ^ 1, abort_flag, DEVERR_SCHEDULE)) break;
+                recs[slot].flags = REC_END;
+                mbar_arrive(smem_u32(&q_full[slot]));
+            }
+        }
+        __syncwarp();
+    } else if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint64_t pol_stream = policy_evict_first();
             const uint64_t pol_keep = policy_evict_last();
-            Piece pc;
-            int32_t t = 0, xb = 0, xcur = 0;
+            int32_t t = 0, xb = 0, wb = 0;
             const uint32_t w_bytes = (uint32_t)(BN * geo.K * 2);
             const uint32_t x_bytes = (uint32_t)(BM * geo.K * geo.x_bytes);
-            while (walk.next(pc)) {
-                if (pc.new_x) {
-                    xcur = xb++;
+            while (true) {
+                const int slot = t % QS;
+                if (!mbar_wait(smem_u32(&q_full[slot]), (t / QS) & 1, abort_flag, DEVERR_TIMEOUT_PRODUCER)) break;
+                const PieceRec pc = recs[slot];
+                mbar_arrive(smem_u32(&q_empty[slot]));
+                if (pc.flags & REC_END) break;
+                if (pc.flags & REC_NEW_X) {
+                    const int32_t xcur = xb++;
                     if (geo.convert_x) {
                         const int s = xcur % SXR;
                         if (!mbar_wait(smem_u32(&xr_empty[s]), ((xcur / SXR) & 1) ^ 1, abort_flag,
@@ -573,9 +535,10 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                                     smem_u32(&xo_full[s]), pol_keep);
                     }
                 }
-                {
-                    const int s = t % SW;
-                    if (!mbar_wait(smem_u32(&w_empty[s]), ((t / SW) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_PRODUCER))
+                if (pc.flags & REC_NEW_W) {
+                    const int32_t wcur = wb++;
+                    const int s = wcur % SW;
+                    if (!mbar_wait(smem_u32(&w_empty[s]), ((wcur / SW) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_PRODUCER))
                         break;
                     mbar_expect_tx(smem_u32(&w_full[s]), w_bytes);
                     for (int b = 0; b < geo.w_nblk; ++b)
@@ -586,20 +549,23 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             }
         }
     } else if (warp == 2) {
-        // ------------------------------------------------------------ ring allocation + output-tile loads
+        // ------------------------------------------------------------ output-tile loads
         if (lane == 0) {
             const uint64_t pol_stream = policy_evict_first();
             int32_t* ends = reinterpret_cast<int32_t*>(smem + geo.off_ends);   // ring head after each piece
-            Piece pc;
-            int32_t t = 0, head = 0, tail_head = 0, tail_piece = 0;
+            int32_t t = 0, tail_head = 0, tail_piece = 0;
             bool ok = true;
-            while (ok && walk.next(pc)) {
+            while (ok) {
+                const int slot = t % QS;
+                if (!mbar_wait(smem_u32(&q_full[slot]), (t / QS) & 1, abort_flag, DEVERR_TIMEOUT_PRODUCER)) break;
+                const PieceRec pc = recs[slot];
+                mbar_arrive(smem_u32(&q_empty[slot]));
+                if (pc.flags & REC_END) break;
                 // whole 8-row groups: in add mode the rows past the piece in its last
                 // group are read but never written back
                 const int rows8 = (pc.rows + GROUP - 1) & ~(GROUP - 1);
-                const int32_t pos = ring_place(head, rows8, R);
                 // free the oldest pieces until this one fits and its barriers are reusable
-                while (tail_piece < t && (head - tail_head > R || t - tail_piece >= RING_PIECES)) {
+                while (tail_piece < t && (pc.head_end - tail_head > R || t - tail_piece >= RING_PIECES)) {
                     const int fi = tail_piece % RING_PIECES;
                     if (!mbar_wait(smem_u32(&y_free[fi]), (tail_piece / RING_PIECES) & 1, abort_flag,
                                    DEVERR_TIMEOUT_PRODUCER)) {
@@ -610,18 +576,17 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     ++tail_piece;
                 }
                 if (!ok) break;
-                ends[t % RING_PIECES] = head;
+                ends[t % RING_PIECES] = pc.head_end;
                 const uint32_t bar = smem_u32(&y_full[t % RING_PIECES]);
                 if (ADD) {
                     const int nch = (pc.ncols + CC - 1) / CC;
                     mbar_expect_tx(bar, (uint32_t)(rows8 * 128 * nch));
                     const uint32_t ring = smem_u32(smem + geo.off_y);
-                    const int32_t xcol0 = pc.col0;
                     for (int c = 0; c < nch; ++c) {
                         for (int r = 0; r < rows8;) {
                             const int k = box_level(rows8 - r, NUM_YMAPS - 1);
-                            tma_load_2d(ring + c * RING_STRIDE + (pos + r) * 128, &ymaps.m[pc.slice][k], xcol0 + c * CC,
-                                        pc.blk_row0 + r, bar, pol_stream);
+                            tma_load_2d(ring + c * RING_STRIDE + (pc.pos + r) * 128, &ymaps.m[pc.slice][k],
+                                        pc.col0 + c * CC, pc.blk_row0 + r, bar, pol_stream);
                             r += GROUP << k;
                         }
                     }
@@ -633,15 +598,20 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ x rounding (mixed dtypes) + MMA
-        Piece pc;
-        int32_t t = 0, xb = 0, xcur = 0;
+        int32_t t = 0, xb = 0, xcur = 0, wb = 0, wcur = 0;
         const uint32_t idesc = instr_desc_mn(w_bf16, BM, BN);
         const int kc_real = geo.K / 8, kc_pad = geo.Kp / 8;
         const bool x_bf16 = p.x_dt == SGMV_BF16;
         constexpr int MAX_KSTEPS = MAX_KP / 16;
         const uint64_t a_rel = smem_desc(0, BM * 16, 128);
-        while (walk.next(pc)) {
-            if (pc.new_x) {
+        while (true) {
+            const int slot = t % QS;
+            if (!warp_wait(smem_u32(&q_full[slot]), (t / QS) & 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
+            const PieceRec pc = recs[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&q_empty[slot]));
+            if (pc.flags & REC_END) break;
+            if (pc.flags & REC_NEW_X) {
                 xcur = xb++;
                 const int xs = xcur % SXO;
                 const int pmask = (1 << x_period_log(pc.rows)) - 1;   // operand row m holds x row m % period
@@ -703,8 +673,11 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 }
             }
             const int xs = xcur % SXO;
-            const int ws = t % SW;
-            if (!warp_wait(smem_u32(&w_full[ws]), (t / SW) & 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
+            if (pc.flags & REC_NEW_W) {
+                wcur = wb++;
+                if (!warp_wait(smem_u32(&w_full[wcur % SW]), (wcur / SW) & 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
+            }
+            const int ws = wcur % SW;
             const int as = t % NUM_ACC;
             if (!warp_wait(smem_u32(&acc_empty[as]), ((t / NUM_ACC) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
             tc_fence_after();
@@ -722,28 +695,27 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     tc_mma(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(&acc_full[as]));
-                tc_commit(smem_u32(&w_empty[ws]));
-                if (pc.last_x) tc_commit(smem_u32(&xo_empty[xs]));
+                if (pc.flags & REC_LAST_W) tc_commit(smem_u32(&w_empty[ws]));
+                if (pc.flags & REC_LAST_X) tc_commit(smem_u32(&xo_empty[xs]));
             }
             __syncwarp();
             ++t;
         }
-    } else {
+    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
         // ------------------------------------------------------------ epilogue
         const int q = warp % 4;                  // TMEM lane quadrant of this warp
         const int grp = (warp - EPI_WARP0) / 4;  // this warp's group takes pieces t % EPI_GROUPS == grp
         const int r = q * 32 + lane;             // block row of this thread
         const int ri = r % GROUP;
         constexpr bool out_bf16 = OUT_DT == SGMV_BF16;
-        Piece pc;
-        int32_t t = 0, head = 0;
-        while (walk.next(pc)) {
+        for (int32_t t = grp;; t += EPI_GROUPS) {
+            const int slot = t % QS;
+            if (!warp_wait(smem_u32(&q_full[slot]), (t / QS) & 1, abort_flag, DEVERR_TIMEOUT_EPILOGUE)) break;
+            const PieceRec pc = recs[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&q_empty[slot]));
+            if (pc.flags & REC_END) break;
             const int as = t % NUM_ACC;
-            const int32_t pos = ring_place(head, (pc.rows + GROUP - 1) & ~(GROUP - 1), R);
-            if (t % EPI_GROUPS != grp) {   // the other group's piece
-                ++t;
-                continue;
-            }
             if (!warp_wait(smem_u32(&acc_full[as]), (t / NUM_ACC) & 1, abort_flag, DEVERR_TIMEOUT_EPILOGUE)) break;
             tc_fence_after();
             // every warp of the group waits, so that its release of this piece's
@@ -774,7 +746,7 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                     tmem_ld32(taddr + (uint32_t)(c * CC + sub * 32), *reinterpret_cast<uint32_t(*)[32]>(v + sub * 32));
                 tmem_ld_wait();
                 if (valid) {
-                    uint8_t* rowp = ring + c * RING_STRIDE + (pos + pr) * 128;
+                    uint8_t* rowp = ring + c * RING_STRIDE + (pc.pos + pr) * 128;
                     uint4* grow = reinterpret_cast<uint4*>(reinterpret_cast<char*>(p.out) +
                                                            ((int64_t)(pc.blk_row0 + pr) * p.H + col0 + c * CC) *
                                                                OUT_BYTES);
@@ -831,13 +803,13 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             __syncwarp();
             if (lane == 0) {
                 const int32_t xcol0 = (int32_t)col0;
-                const int q_lo = max(lane0, 0), q_full = min(lane0 + 32, full_end);
+                const int row_lo = max(lane0, 0), row_end = min(lane0 + 32, full_end);
                 for (int c = k_copy; c < NCH; c += 1 << pc.rep_log) {
                     if (c * CC >= ncols) break;
-                    for (int rr = q_lo; rr < q_full;) {
-                        const int k = box_level(q_full - rr, 2);
+                    for (int rr = row_lo; rr < row_end;) {
+                        const int k = box_level(row_end - rr, 2);
                         tma_store_2d(&ymaps.m[pc.slice][k], xcol0 + c * CC, pc.blk_row0 + rr,
-                                     smem_u32(ring + c * RING_STRIDE + (pos + rr) * 128));
+                                     smem_u32(ring + c * RING_STRIDE + (pc.pos + rr) * 128));
                         rr += GROUP << k;
                     }
                 }
@@ -847,7 +819,6 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
                 mbar_arrive(smem_u32(&y_free[t % RING_PIECES]));
             }
             __syncwarp();
-            ++t;
         }
         // the stores must have read shared memory before the CTA exits; the
         // writes themselves complete with the grid
@@ -904,19 +875,25 @@ constexpr int PIECE_WEIGHT_FLOOR = 16;
 constexpr int PIECE_FIXED_GROUPS = 0;
 
 // Shared-memory layout: an output ring of at least 4, else 3, 2, 1 whole
-// 128-row pieces, with the deepest B pipeline that leaves it room.  In add
-// mode the ring also holds the old output loaded ahead of the epilogue, and the
-// loads it can keep in flight set the pace: two B stages, the rest for the
-// ring (measured on one B200, us per call, 2 B stages against the deepest
-// that fits: rank-64 MLP 169.4 vs 178.3; QKV prefill and the decode-like mix
-// unchanged; overwrite mode is better with the deep B pipeline).
-inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, bool add, int* total_out) {
+// 128-row pieces, with the deepest B pipeline that leaves it room, after the
+// segment table (and, in the balanced mode, its bucket-sorted index) and the
+// piece queue.  In add mode the ring also holds the old output loaded ahead of
+// the epilogue, and the loads it can keep in flight set the pace: two B
+// stages, the rest for the ring (measured on one B200, us per call, 2 B
+// stages against the deepest that fits: rank-64 MLP 169.4 vs 178.3; QKV
+// prefill and the decode-like mix unchanged; overwrite mode is better with the
+// deep B pipeline).  A segment table too long for a ring of one piece leaves
+// the call to the generic kernel.
+inline bool layout_smem(Geometry& g, int32_t nseg, int32_t out_bytes, bool add, int* total_out) {
     const int sw_deep[] = {8, 6, 4, 3, 2};
     const int sw_two[] = {2};
     const int* sw_opts = add ? sw_two : sw_deep;
     const int n_sw = add ? 1 : 5;
     const int32_t row_bytes = g.bn * out_bytes;            // one ring row across all chunks
     const int num_acc = TMEM_COLS / g.bn;
+    const int32_t seg_bytes = round_up(nseg * (int32_t)sizeof(SegEntry), 16);
+    const int32_t inv_bytes = g.mode == MODE_AUTO && g.spread == sched::MODE_BALANCED ? round_up(nseg * 4, 16) : 0;
+    const int32_t q_bytes = QS * (int32_t)sizeof(PieceRec);
     const int32_t budget = SMEM_OPTIN - SMEM_STATIC_RESERVE - 1024;   // 1024: base alignment slack
     for (int prefer_rows : {4 * BM, 3 * BM, 2 * BM, BM}) {
         for (int si = 0; si < n_sw; ++si) {
@@ -924,9 +901,10 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, bool 
             g.stages_w = sw;
             g.stages_xo = 2;
             g.stages_xr = g.convert_x ? 1 : 0;
-            int32_t fixed = sw * g.w_bytes + g.stages_xo * g.xo_bytes + g.stages_xr * g.xr_bytes +
-                            round_up(seg_bytes, 16) + RING_PIECES * 4 +
-                            8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * num_acc + 2 * RING_PIECES) + 64;
+            const int n_bars = 2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * num_acc + 2 * RING_PIECES + 2 * QS;
+            const int32_t fixed = sw * g.w_bytes + g.stages_xo * g.xo_bytes + g.stages_xr * g.xr_bytes + seg_bytes +
+                                  inv_bytes + RING_PIECES * 4 + q_bytes + 8 * n_bars + 64;
+            if (fixed >= budget) continue;
             const int32_t rows = ((budget - fixed) / row_bytes) & ~(GROUP - 1);
             if (rows < prefer_rows) continue;
             g.ring_rows = rows;
@@ -940,11 +918,15 @@ inline bool layout_smem(Geometry& g, int32_t seg_bytes, int32_t out_bytes, bool 
             g.off_xr = off;
             off += g.stages_xr * g.xr_bytes;
             g.off_seg = off;
-            off += round_up(seg_bytes, 16);
+            off += seg_bytes;
+            g.off_inv = off;
+            off += inv_bytes;
             g.off_ends = off;
             off += RING_PIECES * 4;
+            g.off_q = round_up(off, 16);
+            off = g.off_q + q_bytes;
             g.off_bar = round_up(off, 8);
-            off = g.off_bar + 8 * (2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * num_acc + 2 * RING_PIECES);
+            off = g.off_bar + 8 * n_bars;
             const int total = off + 1024;
             if (total > SMEM_OPTIN - SMEM_STATIC_RESERVE) continue;
             *total_out = total;
@@ -964,7 +946,7 @@ inline bool slice_ok(const Problem& p) {
     if (p.lora_num > 1 && ((p.w_as * 2) % 16 || p.w_as < p.N * p.w_ns)) return false;
     if (!aligned16(p.x) || !aligned16(p.w) || !aligned16(p.out)) return false;
     if ((p.H * so) % 16 || (p.off * so) % 16 || (p.N * so) % 16) return false;
-    if (p.batches > SEG_CAP) return false;
+    if (p.batches > SEG_CAP) return false;   // the shared-memory layout sets the real limit
     if (p.out_rows >= (int64_t(1) << 31) || p.x_rows >= (int64_t(1) << 31) || p.off + p.N >= (int64_t(1) << 31))
         return false;
     if (p.lora_num >= (int64_t(1) << 31)) return false;
@@ -1012,9 +994,12 @@ inline bool make_plan_bn(const Problem* ps, int nsl, int sm_count, int bn, Plan*
     g.w_is_bf16 = p.w_dt == SGMV_BF16;
     g.wmin = PIECE_WEIGHT_FLOOR;
     g.bn = bn;
-    // Round-robin pieces are allowed unless x must be rounded to the weights'
-    // dtype: that is done once per x block, so a CTA keeps a block's n-tiles.
-    g.rr = g.convert_x ? 0 : 1;
+    // Pieces dealt across the CTAs (the kernel picks, see choose_mode) unless x
+    // must be rounded to the weights' dtype: that is done once per x block, so
+    // a CTA then takes contiguous pieces and keeps a block across its n-tiles.
+    g.mode = g.convert_x ? (int32_t)sched::MODE_CONTIG : MODE_AUTO;
+    g.spread = sched::MODE_RR;
+    g.halves = 2;
     g.wfix = (int32_t)wfix;
     // B tile: K in blocks of 64 columns, then at most one each of 32, 16, 8
     {
@@ -1059,8 +1044,7 @@ inline bool make_plan_bn(const Problem* ps, int nsl, int sm_count, int bn, Plan*
     }
     g.xo_bytes = BM * g.Kp * 2;
     g.xr_bytes = round_up(BM * (int32_t)p.K * (int32_t)sx, 1024);
-    const int32_t seg_bytes = round_up((int32_t)p.batches * (int32_t)sizeof(SegEntry), 16);
-    if (!layout_smem(g, seg_bytes, (int32_t)so, p.add, &out->smem_bytes)) return false;
+    if (!layout_smem(g, (int32_t)p.batches, (int32_t)so, p.add, &out->smem_bytes)) return false;
 
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;

@@ -7,7 +7,7 @@
 // host too, so that a CPU test can enumerate the pieces of every CTA of a
 // grid and check that together they cover every written element exactly once.
 //
-// Two ways to hand out pieces (the same decision in every CTA):
+// Four ways to hand out pieces (the same decision in every CTA):
 //
 //   balanced   Pieces of full 128-row blocks, in segment order with the n-tile
 //              fastest, are dealt round-robin (CTA c takes c, c + G, ...), so
@@ -19,11 +19,25 @@
 //              of their block (heaviest first: 8-row groups, 16 buckets, a
 //              counting sort) and dealt in snake order (CTA 0, 1, ..., G-1,
 //              G-1, ..., 0, 0, 1, ...), which evens out the CTAs' loads.
+//   round-robin  All pieces, in segment order with the n-tile fastest, dealt
+//              round-robin: the balanced deal without its sorted tail.
 //   contiguous Each CTA takes the pieces that start in its equal share of the
 //              total weight (a piece weighs its 8-row groups, at least a floor,
 //              plus its B tile), in the same order; consecutive pieces of a CTA
 //              then share their x block, which is converted to the weights'
 //              dtype once (used when x's dtype differs from the weights').
+//   dynamic    Round-robin without its last rounds: a launch has G0 + E CTAs, of
+//              which G0 run at once; unit u < G0 is round-robin share u of the
+//              first H pieces (whole rounds, all but the last few), unit
+//              G0 + e is chunk e of the rest, cut into E near-equal runs of
+//              consecutive pieces.  A CTA processes its own unit, then claims
+//              units whose CTAs have not started (cluster launch control, in
+//              the kernel) until none is left, so the end of the launch is
+//              shared out by how fast each SM actually drains its pieces.
+//   columns    Each CTA takes an equal share of the pieces counted in segment
+//              order with the row block fastest within each n-tile, so that
+//              consecutive pieces of a CTA share their B tile (the adapter's
+//              n-tile stays staged while x blocks stream past it).
 #pragma once
 
 #include <stdint.h>
@@ -43,13 +57,16 @@ constexpr int GROUPS_PER_BLOCK = BM / GROUP;
 constexpr int MAX_SLICES = 4;
 constexpr int NUM_BUCKETS = 16;         // a partial block's 8-row groups: 1..16
 
-enum : int32_t { MODE_CONTIG = 0, MODE_BALANCED = 1 };
+enum : int32_t { MODE_CONTIG = 0, MODE_BALANCED = 1, MODE_RR = 2, MODE_COLS = 3, MODE_DYNAMIC = 4 };
+
+constexpr int DYN_TAIL_ROUNDS = 3;      // dynamic mode: whole round-robin rounds left to the claimed chunks
 
 struct SegEntry {
     int32_t row0;
     int32_t rows;       // 0: the segment writes nothing (guards applied)
     int32_t adapter;
-    int32_t prefix;     // balanced: full-block pieces of earlier segments; contiguous: their weight
+    int32_t prefix;     // balanced: full-block pieces of earlier segments; round-robin and columns:
+                        // all their pieces; contiguous: their weight
 };
 
 // The slices of one launch: slice s covers output columns [off[s], off[s] + N[s])
@@ -76,6 +93,7 @@ SGMV_HD int32_t imax(int32_t a, int32_t b) { return a > b ? a : b; }
 
 // Units of one segment in the scan that fills SegEntry::prefix.
 SGMV_HD int32_t full_pieces(int32_t rows, int32_t n_tiles) { return rows / BM * n_tiles; }
+SGMV_HD int32_t all_pieces(int32_t rows, int32_t n_tiles) { return (rows + BM - 1) / BM * n_tiles; }
 SGMV_HD int32_t contig_weight(int32_t rows, int32_t n_tiles, int32_t wmin, int32_t wfix) {
     const int32_t G = (rows + GROUP - 1) / GROUP;
     if (G == 0) return 0;
@@ -142,10 +160,36 @@ struct Gen {
     // balanced: head (round-robin over full pieces) then tail items
     int32_t hs, hloc, f;          // head: segment, piece within its full pieces, global index
     int32_t m, which;             // tail: round and item of the round
+    int32_t rr_end;               // round-robin: all pieces
+    int32_t cend;                 // columns: end of this CTA's pieces (global; hs, hloc and f walk them)
+    int32_t G0, E, Hd;            // dynamic: CTAs that run at once, chunks, pieces dealt round-robin
     // contiguous walk
     int32_t i, rb, j, cur, w_end, nblk, gcw, wmin, wfix;
 
-    SGMV_HD int32_t fullp(int32_t s) const { return full_pieces(segs[s].rows, n_tiles); }
+    // dynamic mode: the pieces of unit u (its own CTA's, or one it claimed)
+    SGMV_HD void init_unit(int32_t u) {
+        hs = 0;
+        hloc = 0;
+        if (u < G0) {                 // round-robin share u of the first Hd pieces
+            c = u;
+            G = G0;
+            f = u;
+            rr_end = Hd;
+            cend = -1;
+            head_advance(u);
+        } else {                      // chunk u - G0 of the remaining pieces, in order
+            const int32_t e = u - G0, T = tl_total - Hd;
+            f = Hd + (int32_t)(((int64_t)T * e) / E);
+            cend = Hd + (int32_t)(((int64_t)T * (e + 1)) / E);
+            head_advance(f);
+        }
+    }
+    int32_t tl_total;             // dynamic: all pieces
+
+    // pieces of segment s that are dealt round-robin
+    SGMV_HD int32_t fullp(int32_t s) const {
+        return mode == MODE_BALANCED ? full_pieces(segs[s].rows, n_tiles) : all_pieces(segs[s].rows, n_tiles);
+    }
 
     // The piece of block rb of segment s, n-tile j, column half h (h < 0: whole tile).
     // False if the half holds no columns.
@@ -261,13 +305,26 @@ struct Gen {
     }
 
     // ------------------------------------------------------------ interface
-    // total: full pieces (balanced) or total weight (contiguous).
+    // total: full pieces (balanced), all pieces (round-robin) or total weight (contiguous).
     SGMV_HD void init(int32_t cta, int32_t grid, int32_t total, int32_t wmin_, int32_t wfix_) {
         c = cta;
         G = grid;
         wmin = wmin_;
         wfix = wfix_;
-        if (mode == MODE_BALANCED) {
+        rr_end = total;
+        if (mode == MODE_DYNAMIC) {
+            tl_total = total;
+            G0 = grid;                // grid: the CTAs that run at once (the caller passes G0)
+            const int32_t rounds = total / G0 - DYN_TAIL_ROUNDS;
+            Hd = rounds > 0 ? rounds * G0 : 0;
+            init_unit(cta);
+        } else if (mode == MODE_COLS) {
+            f = (int32_t)(((int64_t)total * c) / G);
+            cend = (int32_t)(((int64_t)total * (c + 1)) / G);
+            hs = 0;
+            hloc = 0;
+            head_advance(f);
+        } else if (mode != MODE_CONTIG) {
             hs = 0;
             hloc = 0;
             f = c;
@@ -280,13 +337,36 @@ struct Gen {
     }
 
     SGMV_HD bool next(Piece& p) {
-        if (mode == MODE_BALANCED) {
-            while (f < tl->H) {
+        if (mode == MODE_DYNAMIC) {
+            if (cend < 0) {           // a round-robin share
+                if (f >= rr_end) return false;
+                make(hs, hloc / n_tiles, hloc % n_tiles, -1, p);
+                f += G;
+                head_advance(G);
+                return true;
+            }
+            if (f >= cend) return false;
+            make(hs, hloc / n_tiles, hloc % n_tiles, -1, p);
+            ++f;
+            head_advance(1);
+            return true;
+        }
+        if (mode == MODE_COLS) {
+            if (f >= cend) return false;
+            const int32_t nblk_s = (segs[hs].rows + BM - 1) / BM;   // row blocks of the segment: the fastest index
+            make(hs, hloc % nblk_s, hloc / nblk_s, -1, p);
+            ++f;
+            head_advance(1);
+            return true;
+        }
+        if (mode != MODE_CONTIG) {
+            while (f < (mode == MODE_RR ? rr_end : tl->H)) {
                 const bool ok = make(hs, hloc / n_tiles, hloc % n_tiles, -1, p);
                 f += G;
                 head_advance(G);
                 if (ok) return true;
             }
+            if (mode == MODE_RR) return false;
             while (true) {   // tail items c + 2Gm and 2G - 1 - c + 2Gm, in increasing order
                 const int32_t it = which == 0 ? c + 2 * G * m : 2 * G - 1 - c + 2 * G * m;
                 if (which == 0) which = 1;

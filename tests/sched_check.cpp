@@ -1,7 +1,7 @@
 // Host check of the tensor-core kernel's piece scheduler (csrc/tc_sched.cuh).
 //
 // For many random segment tables, slice sets, tile widths, grid sizes and
-// both ways of handing out pieces, it enumerates the pieces of every CTA with
+// every way of handing out pieces, it enumerates the pieces of every CTA with
 // the same generator the kernel's scheduler warp runs, and checks that
 // together they write every (row, column) of every valid segment's slices
 // exactly once and nothing else.  It also reports the largest CTA load over
@@ -31,7 +31,7 @@ struct Case {
     int64_t T, A;
     int nsl;
     int64_t off[MAX_SLICES], N[MAX_SLICES];
-    int bn, grid, mode, halves;
+    int bn, grid, mode, halves, dyn_chunks;
 };
 
 static int failures = 0;
@@ -73,6 +73,7 @@ static double run_case(const Case& k) {
     for (int32_t b = 0; b < nseg; ++b) {
         segs[b].prefix = total;
         total += k.mode == MODE_BALANCED ? full_pieces(segs[b].rows, n_tiles)
+                 : k.mode == MODE_RR || k.mode == MODE_COLS || k.mode == MODE_DYNAMIC ? all_pieces(segs[b].rows, n_tiles)
                                          : contig_weight(segs[b].rows, n_tiles, wmin, wfix);
     }
     Tail tl;
@@ -87,7 +88,13 @@ static double run_case(const Case& k) {
     for (int i = 0; i < k.nsl; ++i) H = H > k.off[i] + k.N[i] ? H : k.off[i] + k.N[i];
     std::vector<uint8_t> cover((size_t)k.T * (size_t)H, 0);
     std::vector<double> load(k.grid, 0.0);
-    for (int32_t c = 0; c < k.grid; ++c) {
+    // dynamic mode: the grid has k.grid + E CTAs; each of the first k.grid takes its own unit, then
+    // the remaining units are claimed in an arbitrary order by arbitrary CTAs (here: a shuffled deal)
+    const int32_t E = k.mode == MODE_DYNAMIC ? k.dyn_chunks : 0;
+    std::vector<int32_t> owner(k.grid + E);
+    for (int32_t u = 0; u < k.grid + E; ++u) owner[u] = u < k.grid ? u : (int32_t)uni(0, k.grid - 1);
+    for (int32_t u = 0; u < k.grid + E; ++u) {
+        const int32_t c = owner[u];
         Gen g;
         g.segs = segs.data();
         g.st = &st;
@@ -97,7 +104,14 @@ static double run_case(const Case& k) {
         g.n_tiles = n_tiles;
         g.bn = k.bn;
         g.mode = k.mode;
-        g.init(c, k.grid, total, wmin, wfix);
+        if (k.mode == MODE_DYNAMIC) {
+            g.E = E;
+            g.init(u < k.grid ? u : 0, k.grid, total, wmin, wfix);
+            if (u >= k.grid) g.init_unit(u);
+        } else {
+            if (u >= k.grid) break;
+            g.init(c, k.grid, total, wmin, wfix);
+        }
         Piece p;
         int guard = 0;
         while (g.next(p)) {
@@ -167,7 +181,8 @@ static Case random_case(int shape) {
         col += N;
     }
     k.grid = (int)(uni(0, 2) == 0 ? uni(1, 9) : uni(0, 1) ? 148 : uni(10, 200));
-    k.mode = uni(0, 1) ? MODE_BALANCED : MODE_CONTIG;
+    k.mode = (int)uni(0, 4);   // MODE_CONTIG, MODE_BALANCED, MODE_RR, MODE_COLS or MODE_DYNAMIC
+    k.dyn_chunks = (int)uni(1, 3 * k.grid);
     k.halves = uni(0, 1) ? 2 : 1;
     return k;
 }
@@ -188,6 +203,7 @@ int main(int argc, char** argv) {
     // The round-robin-plus-sorted-tail deal on a QKV-like batch: 16 segments of 64..1024 rows,
     // 2 of them idle, three 4096-column slices, 148 CTAs.
     {
+        rng_state = 0x2545F4914F6CDD1Dull;   // a fixed batch, whatever the random cases drew
         Case k;
         int64_t row = 0;
         for (int b = 0; b < 16; ++b) {
@@ -205,6 +221,7 @@ int main(int argc, char** argv) {
         k.bn = 128;
         k.grid = 148;
         k.mode = MODE_BALANCED;
+        k.dyn_chunks = 0;
         for (int hv : {1, 2}) {
             k.halves = hv;
             const double r = run_case(k);

@@ -373,6 +373,33 @@ def test_more_pieces_per_cta_than_ring_slots(case, variant):
     assert pieces > 32 * torch.cuda.get_device_properties(0).multi_processor_count
 
 
+@pytest.mark.parametrize("variant", ["auto", "tc_wide"])
+def test_thousands_of_segments_take_the_tensor_cores(variant):
+    """4096 segments (short, full-block and longer ones mixed, ids -1 and out of range among them): the
+    segment table stays in shared memory, the tensor-core kernel takes the call and every element
+    matches the oracle."""
+    rng = np.random.default_rng(4096)
+    B = 4096
+    kind = rng.random(B)
+    lengths = np.where(kind < 0.6, rng.integers(1, 41, B), np.where(kind < 0.8, 128, rng.integers(129, 301, B)))
+    idx = rng.integers(-1, 17, B)                 # 16 is out of range: skipped like -1
+    p = gen.custom(seed=96, lengths=lengths.tolist(), K=16, N=256, H=512, offset=128, num_adapters=16,
+                   idx=idx.tolist())
+    dp = DeviceProblem(p)
+    if variant == "auto":
+        sg.set_variant(sg.VARIANT_AUTO)
+        assert dp.plan() == sg.VARIANT_TC
+    else:
+        assert use_variant(variant, dp)
+    dp.run()
+    torch.cuda.synchronize()
+    assert sg.device_error() == 0
+    gpu = dp.result()
+    ref = oracle.run_problem(p, nthreads=oracle.max_threads())
+    err, count = compare_every_element(gpu, ref, p, regions(p))
+    report(f"segments_4096/{variant}", compared=count, max_abs_err=err)
+
+
 # ------------------------------------------------------------------ metadata validation
 
 def test_validate_metadata_bits():

@@ -11,7 +11,7 @@ import torch
 import oracle
 import sgmv_inputs as gen
 import segmented_gather_gemm_expand_b200 as sg
-from sgmv_testlib import compare, from_torch, to_torch
+from sgmv_testlib import compare, compare_every_element, from_torch, report, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -104,7 +104,8 @@ def test_shrink_hidden_sizes(H):
 
 
 def test_shrink_qkv_prefill_sized():
-    """The shrink that feeds the fused-QKV prefill batch: 16 sequences U[64,1024], hidden 4096, rank 16."""
+    """The shrink that feeds the fused-QKV prefill batch: 16 sequences U[64,1024], hidden 4096, rank 16.
+    A prefill batch takes the row-balanced kernel: one launch, no workspace, no H split."""
     rng = np.random.default_rng(0)
     lengths = rng.integers(64, 1025, 16)
     idx = rng.integers(0, 32, 16)
@@ -112,4 +113,68 @@ def test_shrink_qkv_prefill_sized():
     p = shrink_problem(8, lengths.tolist(), H=4096, R=16, A=32, idx=idx.tolist(), out_dt="bf16")
     import oracle as o
     v, splits, _ = run_shrink(p, nthreads=o.max_threads())
-    assert v == sg.VARIANT_TC and splits > 1
+    assert v == sg.VARIANT_TC and splits == 1
+
+
+# ---------------------------------------------------------------- the row-balanced kernel
+
+def row_balanced_check(p, name):
+    """Run sgmv_shrink on a prefill-sized batch, assert that the row-balanced kernel took it (no
+    workspace wanted at any size), and compare every element with the oracle's shrink."""
+    c = p.calls[0]
+    x, a, y = to_torch(p.x, p.x_dt), to_torch(c.w, p.w_dt), to_torch(p.y0, p.out_dt)
+    meta = [torch.as_tensor(np.asarray(m)).cuda() for m in (p.seq_start, p.seq_len, p.lora_idx)]
+    v, splits, pref = sg.shrink_plan(x, a, y, *meta, p.batches, p.max_seq_len, 1 << 30)
+    assert v == sg.VARIANT_TC and splits == 1 and pref == 0, (v, splits, pref)
+    sg.sgmv_shrink(x, a, y, *meta, p.batches, p.max_seq_len)
+    torch.cuda.synchronize()
+    assert sg.device_error() == 0
+    gpu = from_torch(y, p.out_dt)
+    ref = oracle.shrink(p.x, p.x_dt, c.w, p.w_dt, p.y0, p.out_dt, p.seq_start, p.seq_len, p.lora_idx,
+                        nthreads=oracle.max_threads())
+    rows = np.zeros(p.y0.shape[0], dtype=bool)
+    lim = min(p.y0.shape[0], p.x.shape[0])
+    for s_, L, ai in zip(p.seq_start, p.seq_len, p.lora_idx):
+        if 0 <= ai < c.w.shape[0] and s_ >= 0 and L > 0:
+            rows[s_:min(s_ + L, lim)] = True
+    err, count = compare_every_element(gpu, ref, p, [(rows, 0, c.w.shape[-2])])
+    assert count == int(rows.sum()) * c.w.shape[-2]
+    report(f"shrink_rows/{name}", compared=count, max_abs_err=err)
+    # the same call twice gives the same bits (one CTA sums each row, in chunk order)
+    y2 = to_torch(p.y0, p.out_dt)
+    sg.sgmv_shrink(x, a, y2, *meta, p.batches, p.max_seq_len)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_torch(y2, p.out_dt), gpu)
+
+
+ROW_CASES = {
+    # lengths, hidden, rank, adapters, extra keywords
+    "rank16_bf16": dict(lengths=[700, 0, 1300, 64, 5, 900, 33], H=4096, R=16, A=4, idx=[0, 1, 2, -1, 3, 1, 2],
+                        out_dt="bf16"),
+    "rank32_f32_out": dict(lengths=[1000, 1500, 77], H=1000, R=32, A=3, out_dt="f32"),
+    "rank64_f16": dict(lengths=[2000, 600], H=520, R=64, A=2, x_dt="f16", w_dt="f16", out_dt="f16"),
+    "rank128": dict(lengths=[1200, 1300], H=256, R=128, A=2, out_dt="f32"),
+    "short_segments_two_per_tile": dict(lengths=[40, 36, 45, 9] * 20, H=512, R=16, A=5, out_dt="bf16"),
+    "tiles_of_128_rows": dict(lengths=[5000, 4000, 3000, 1], H=384, R=16, A=3, out_dt="bf16"),
+    "gaps_invalid_ids_rows_past_out": dict(lengths=[900, 800, 700, 600], starts=[3, 1000, 1900, 2650], H=640,
+                                           R=16, A=2, idx=[0, 5, 1, -1], extra_rows=7, out_dt="f32"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(ROW_CASES))
+def test_shrink_row_balanced(case):
+    kw = dict(ROW_CASES[case])
+    p = shrink_problem(len(case), **kw)
+    row_balanced_check(p, case)
+
+
+def test_shrink_row_balanced_out_shorter_than_x():
+    """Rows at or past the output's row count are skipped (the output has fewer rows than x)."""
+    p = shrink_problem(9, [1500, 1500], H=512, R=16, A=2, out_dt="bf16")
+    p.y0 = np.ascontiguousarray(p.y0[:2800])
+    row_balanced_check(p, "out_shorter_than_x")
+
+
+def test_shrink_workload_every_element():
+    """The qkv_shrink workload (the bench's shrink line) at full size, every element."""
+    row_balanced_check(gen.WORKLOADS["qkv_shrink"](), "qkv_shrink")

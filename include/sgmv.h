@@ -237,15 +237,11 @@ SGMV_API int bgmv_expand_slice(const sgmv_tensor* inputs, const sgmv_tensor* lor
  *             keep their bits
  *   workspace, workspace_bytes  optional DEVICE scratch (16-byte aligned, else
  *             SGMV_ERR_WORKSPACE), owned by the caller and used only by the
- *             work this call enqueues.  Prefill batches (at least 16 rows per
- *             SM and 32 rows per segment on average) need none: one launch
- *             hands every SM an equal share of the rows, in 8-row groups, and
- *             sums each row over the whole hidden size in one CTA
- *             (deterministic).  Other batches, with a workspace, split H into
- *             up to 16 parts (the count a cost model of the busiest SM's
- *             bytes and per-item pipeline work prefers, halved until the
- *             partial sums fit) and add the fp32 partial sums in a second
- *             kernel, in a fixed order (deterministic); without one (NULL or
+ *             work this call enqueues.  With it the tensor-core kernel splits
+ *             H into up to 16 parts (the count a cost model of the busiest
+ *             SM's bytes and per-item pipeline work prefers, halved until the
+ *             partial sums fit) and adds the fp32 partial sums in a second
+ *             kernel, in a fixed order (deterministic); without it (NULL or
  *             too small for two parts) each row block is one work item.
  *             Calls that run at the same time need separate workspaces.
  *

@@ -28,7 +28,6 @@ __device__ void raise_device_error(int32_t bits) { atomicOr(&g_device_error, bit
 
 #include "tc_kernel.cuh"
 #include "shrink.cuh"
-#include "shrink_rows.cuh"
 
 static_assert(SGMV_MAX_SLICES == sgmv::tc::MAX_SLICES, "one fused launch takes every slice of a call");
 
@@ -360,10 +359,7 @@ int validate_shrink(const sgmv_tensor* x, const sgmv_tensor* a, const sgmv_tenso
     return SGMV_OK;
 }
 
-// Variant and split count of a validated, non-empty shrink call with the given
-// workspace.  Prefill batches run the row-balanced kernel (one launch, whole
-// hidden size per row, no workspace: *splits = 1); others split H when a
-// workspace holds the partial sums.
+// Variant and split count of a validated, non-empty shrink call with the given workspace.
 int choose_shrink(const Call& c, const DeviceInfo& dev, int forced, const void* ws, size_t ws_bytes, int* splits) {
     *splits = 1;
     const bool tc_ok = dev.cc_major == 10 && shr::supports(c.p) && c.p.batches <= shr::SEG_CAP;
@@ -373,7 +369,7 @@ int choose_shrink(const Call& c, const DeviceInfo& dev, int forced, const void* 
     else if (forced == SGMV_VARIANT_TC || forced == SGMV_VARIANT_TC_WIDE)
         v = tc_ok ? (int)SGMV_VARIANT_TC : (int)SGMV_ERR_VARIANT;
     else v = tc_ok ? SGMV_VARIANT_TC : SGMV_VARIANT_SIMT;
-    if (v == SGMV_VARIANT_TC && ws && !shr::rows_kernel_fits(c.p, dev.sm_count)) {
+    if (v == SGMV_VARIANT_TC && ws) {
         int sp = shr::preferred_splits(c.p, dev.sm_count);
         while (sp > 1 && (size_t)shr::workspace_bytes_for(c.p, sp) > ws_bytes) sp /= 2;
         *splits = sp;
@@ -382,15 +378,6 @@ int choose_shrink(const Call& c, const DeviceInfo& dev, int forced, const void* 
 }
 
 int launch_shrink(const Call& c, const DeviceInfo& dev, int splits, float* ws, cudaStream_t stream) {
-    if (shr::rows_kernel_fits(c.p, dev.sm_count)) {
-        shr::RowPlan rp;
-        if (!shr::make_rows_plan(c.p, dev.sm_count, tc::encode_fn(), &rp)) return SGMV_ERR_VARIANT;
-        switch (c.p.out_dt) {
-            case SGMV_F32: return shr::launch_rows_dt<SGMV_F32>(rp, c.p, stream);
-            case SGMV_BF16: return shr::launch_rows_dt<SGMV_BF16>(rp, c.p, stream);
-            default: return shr::launch_rows_dt<SGMV_F16>(rp, c.p, stream);
-        }
-    }
     shr::Plan pl;
     if (!shr::make_plan(c.p, dev.sm_count, splits, tc::encode_fn(), &pl)) return SGMV_ERR_VARIANT;
     switch (c.p.out_dt) {
@@ -502,7 +489,7 @@ int sgmv_shrink_plan(const sgmv_tensor* inputs, const sgmv_tensor* lora_a, const
     if (v < 0) return v;
     *variant = v;
     *splits = v == SGMV_VARIANT_TC ? sp : 1;
-    if (v == SGMV_VARIANT_TC && !shr::rows_kernel_fits(c.p, dev.sm_count))
+    if (v == SGMV_VARIANT_TC)
         *preferred_workspace_bytes = (size_t)shr::workspace_bytes_for(c.p, shr::preferred_splits(c.p, dev.sm_count));
     return SGMV_OK;
 }

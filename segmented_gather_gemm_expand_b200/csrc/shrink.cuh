@@ -15,8 +15,12 @@
 // in split order (deterministic) and rounds into out.
 //
 // One CTA per SM, 192 threads: warp 0 TMA producer, warp 1 MMA, warps 2-5
-// epilogue.  Items are handed out round-robin.  Every mbarrier wait is
-// bounded and reports a timeout through the device error word.
+// epilogue.  Items are handed out round-robin, the items of full 128-row
+// blocks first and those of the segments' partial last blocks after them, so
+// that the last, incomplete round of the deal holds the smaller items
+// (measured on the QKV shrink: 21.5 against 22.3 us with segment order).
+// Every mbarrier wait is bounded and reports a timeout through the device
+// error word.
 #pragma once
 
 #include <cuda.h>
@@ -39,7 +43,9 @@ constexpr int MAX_RANK = 128;
 constexpr int SMEM_LIMIT = 232448 - 1024;   // dynamic shared memory a CTA may opt in to on sm_100
 
 struct SegRow {
-    int32_t row0, rows, adapter, prefix;   // prefix: row blocks of earlier segments
+    int32_t row0, rows, adapter;
+    int32_t prefix;    // full 128-row blocks of earlier segments
+    int32_t pprefix;   // earlier segments that end in a partial block
 };
 
 struct Geo {
@@ -62,17 +68,23 @@ struct Item {
 };
 
 // Item `id` of the round-robin sequence: block id / splits, split id % splits.
-__device__ __forceinline__ void decode_item(const SegRow* segs, int32_t nseg, const Geo& g, int32_t id, Item& it) {
+// Blocks are numbered full ones first (segment order), then every segment's
+// partial last block: the last, incomplete round of the deal then holds the
+// smaller items, which evens out the CTAs' work.  full_blocks: all full blocks.
+__device__ __forceinline__ void decode_item(const SegRow* segs, int32_t nseg, const Geo& g, int32_t full_blocks,
+                                            int32_t id, Item& it) {
     const int32_t blk = id / g.splits;
     it.split = id - blk * g.splits;
-    int lo = 0, hi = nseg - 1;   // last segment whose prefix <= blk (empty segments share their successor's)
+    const bool partial = blk >= full_blocks;
+    const int32_t key = partial ? blk - full_blocks : blk;
+    int lo = 0, hi = nseg - 1;   // last segment whose prefix <= key (empty ones share their successor's)
     while (lo < hi) {
         const int mid = (lo + hi + 1) / 2;
-        if (segs[mid].prefix <= blk) lo = mid;
+        if ((partial ? segs[mid].pprefix : segs[mid].prefix) <= key) lo = mid;
         else hi = mid - 1;
     }
     const SegRow s = segs[lo];
-    const int32_t rb = blk - s.prefix;
+    const int32_t rb = partial ? s.rows / BM : key - s.prefix;
     it.row0 = s.row0 + rb * BM;
     it.rows = min(BM, s.rows - rb * BM);
     it.adapter = s.adapter;
@@ -93,7 +105,7 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ int s_abort;
     __shared__ uint32_t s_tmem_base;
-    __shared__ int32_t s_total_blocks;
+    __shared__ int32_t s_total_blocks, s_full_blocks;
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     SegRow* segs = reinterpret_cast<SegRow*>(smem + g.off_seg);
@@ -128,28 +140,41 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
     // grid to finish before it reads the partial sums.
     grid_dependents_launch();
 
-    // Segment table (guards of sgmv.h applied) and the prefix of row blocks.
+    // Segment table (guards of sgmv.h applied), the prefix of full row blocks
+    // and the count of partial last blocks before each segment.
     const int32_t nseg = (int32_t)p.batches;
     for (int32_t b = tid; b < nseg; b += THREADS) {
         const Segment s = load_segment(p, b);
-        segs[b] = SegRow{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0};
+        segs[b] = SegRow{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0, 0};
     }
     __syncthreads();
     if (warp == 0) {
-        int32_t running = 0;
+        int32_t run_full = 0, run_part = 0;
         for (int32_t base = 0; base < nseg; base += 32) {
             const int32_t b = base + lane;
-            const int32_t blocks = b < nseg ? (segs[b].rows + BM - 1) / BM : 0;
-            int32_t v = blocks;
+            const int32_t full = b < nseg ? segs[b].rows / BM : 0;
+            const int32_t part = b < nseg ? (segs[b].rows % BM != 0) : 0;
+            int32_t v = full, w = part;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += t;
+                const int32_t u = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) {
+                    v += t;
+                    w += u;
+                }
             }
-            if (b < nseg) segs[b].prefix = running + v - blocks;
-            running += __shfl_sync(0xffffffffu, v, 31);
+            if (b < nseg) {
+                segs[b].prefix = run_full + v - full;
+                segs[b].pprefix = run_part + w - part;
+            }
+            run_full += __shfl_sync(0xffffffffu, v, 31);
+            run_part += __shfl_sync(0xffffffffu, w, 31);
         }
-        if (lane == 0) s_total_blocks = running;
+        if (lane == 0) {
+            s_full_blocks = run_full;
+            s_total_blocks = run_full + run_part;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -157,6 +182,7 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
 
     const uint32_t tmem_base = s_tmem_base;
     const int32_t n_items = s_total_blocks * g.splits;
+    const int32_t full_blocks = s_full_blocks;
     volatile int* abort_flag = &s_abort;
     const bool bf16 = p.w_dt == SGMV_BF16;
 
@@ -169,7 +195,7 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
             Item it;
             bool ok = true;
             for (int32_t id = blockIdx.x; ok && id < n_items; id += gridDim.x) {
-                decode_item(segs, nseg, g, id, it);
+                decode_item(segs, nseg, g, full_blocks, id, it);
                 const int rows8 = (it.rows + 7) & ~7;
                 for (int32_t ch = it.ch0; ch < it.ch1; ++ch, ++q) {
                     const uint32_t s = q % S;
@@ -194,7 +220,7 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
         uint32_t q = 0, n = 0;
         Item it;
         for (int32_t id = blockIdx.x; id < n_items; id += gridDim.x, ++n) {
-            decode_item(segs, nseg, g, id, it);
+            decode_item(segs, nseg, g, full_blocks, id, it);
             const uint32_t acc = n % NUM_ACC;
             if (!warp_wait(smem_u32(&acc_empty[acc]), ((n / NUM_ACC) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
             tc_fence_after();
@@ -230,7 +256,7 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
         uint32_t n = 0;
         Item it;
         for (int32_t id = blockIdx.x; id < n_items; id += gridDim.x, ++n) {
-            decode_item(segs, nseg, g, id, it);
+            decode_item(segs, nseg, g, full_blocks, id, it);
             const uint32_t acc = n % NUM_ACC;
             if (!warp_wait(smem_u32(&acc_full[acc]), (n / NUM_ACC) & 1, abort_flag, DEVERR_TIMEOUT_EPILOGUE)) break;
             tc_fence_after();

@@ -36,10 +36,12 @@
 //                        registers, so nothing outside the segment's rows is
 //                        written.
 //
-// A piece is (segment, 128-row block of the segment, columns of one n-tile or
-// of half of one); how pieces are handed out to CTAs is described in
-// tc_sched.cuh.  Every wait on an mbarrier is bounded; a wait that gives up
-// sets the device error word and makes the CTA leave its loops.
+// A piece is (segment, 128-row block of the segment, one n-tile of columns);
+// how pieces are handed out to CTAs is described in tc_sched.cuh.  Records
+// carry x-block and B-tile reuse flags, so that consecutive pieces of a CTA
+// that share either keep it staged.  Every wait on an mbarrier is bounded; a
+// wait that gives up sets the device error word and makes the CTA leave its
+// loops.
 #pragma once
 
 #include <cuda.h>
@@ -93,8 +95,6 @@ struct Geometry {
     int32_t w_is_bf16;
     int32_t wmin, wfix; // contiguous mode: weight of a piece = max(its 8-row groups, wmin) + wfix
     int32_t mode;       // sched::MODE_CONTIG, or MODE_AUTO: the kernel picks (choose_mode)
-    int32_t spread;     // MODE_AUTO's choice for batches of mostly full blocks: MODE_RR or MODE_BALANCED
-    int32_t halves;     // balanced mode: 2 = the tail is dealt in column halves
     int32_t bn;         // columns per n-tile: 128 or 256 (the kernel's BN)
     // B tile: K split into blocks of 64/32/16/8 columns, each its own TMA box
     // (rows of 2*kb bytes, swizzled by the row width) at w_blk_off in a stage
@@ -108,7 +108,7 @@ struct Geometry {
     uint32_t b_off[MAX_KP / 16];
 
     // shared memory offsets (bytes, from the 1024-aligned base)
-    int32_t off_y, off_w, off_xo, off_xr, off_seg, off_inv, off_ends, off_q, off_bar;
+    int32_t off_y, off_w, off_xo, off_xr, off_seg, off_ends, off_q, off_bar;
     int32_t w_bytes, xo_bytes, xr_bytes;
 };
 
@@ -206,55 +206,21 @@ __device__ int32_t scan_segments(SegEntry* segs, int32_t nseg, int32_t* warp_sum
     return running;
 }
 
-// Segment units of the scan: full-block pieces (balanced), all pieces (round-robin) or weight (contiguous).
+// Segment units of the scan: pieces (round-robin) or weight (contiguous).
 __device__ __forceinline__ int32_t seg_units(const Geometry& geo, int32_t mode, int32_t rows) {
-    if (mode == sched::MODE_BALANCED) return sched::full_pieces(rows, geo.n_tiles);
-    if (mode == sched::MODE_RR || mode == sched::MODE_COLS) return sched::all_pieces(rows, geo.n_tiles);
+    if (mode == sched::MODE_RR) return sched::all_pieces(rows, geo.n_tiles);
     return sched::contig_weight(rows, geo.n_tiles, geo.wmin, geo.wfix);
 }
 
 // How this launch hands out pieces (the same in every CTA).  A batch whose row
 // blocks are mostly partial (short segments: decode-like mixes) takes
 // contiguous ranges, which keep each x block and walk one adapter's B tiles in
-// order; others take geo.spread (their pieces are dealt across the CTAs).
+// order; others are dealt round-robin.  Measured on one B200 (us per call,
+// round-robin vs contiguous): QKV prefill 30.7 vs 32.2, single-tenant 51.4 vs
+// 54.4, decode-like mix 71.5 vs 52.0.
 __device__ __forceinline__ int32_t choose_mode(const Geometry& geo, int32_t partial_blocks, int32_t blocks) {
     if (geo.mode != MODE_AUTO) return geo.mode;
-    return 2 * partial_blocks > blocks ? (int32_t)sched::MODE_CONTIG : geo.spread;
-}
-
-// The sorted tail of the balanced mode, built by the scheduler warp: bucket
-// counts and the segments of each bucket in index order (ballots over chunks
-// of 32 segments, so every CTA builds the same table).
-__device__ void build_tail(const SegEntry* segs, int32_t nseg, int32_t total, int32_t n_tiles, int32_t halves,
-                           sched::Tail* tl, int32_t* inv) {
-    const int lane = threadIdx.x % 32;
-    const uint32_t lt = (1u << lane) - 1u;
-    int32_t cnt[sched::NUM_BUCKETS + 1];
-#pragma unroll
-    for (int r = 0; r <= sched::NUM_BUCKETS; ++r) cnt[r] = 0;
-    for (int32_t base = 0; base < nseg; base += 32) {
-        const int32_t s = base + lane;
-        const int32_t r = s < nseg ? sched::partial_bucket(segs[s].rows) : 0;
-#pragma unroll
-        for (int q = 1; q <= sched::NUM_BUCKETS; ++q) cnt[q] += __popc(__ballot_sync(0xffffffffu, r == q));
-    }
-    sched::Tail t;
-    sched::tail_layout(t, cnt, total, (int32_t)gridDim.x, n_tiles, halves);
-    int32_t fill[sched::NUM_BUCKETS + 1];
-#pragma unroll
-    for (int q = 0; q <= sched::NUM_BUCKETS; ++q) fill[q] = q ? t.seg0[q] : 0;
-    for (int32_t base = 0; base < nseg; base += 32) {
-        const int32_t s = base + lane;
-        const int32_t r = s < nseg ? sched::partial_bucket(segs[s].rows) : 0;
-#pragma unroll
-        for (int q = 1; q <= sched::NUM_BUCKETS; ++q) {
-            const uint32_t m = __ballot_sync(0xffffffffu, r == q);
-            if (r == q) inv[fill[q] + __popc(m & lt)] = s;
-            fill[q] += __popc(m);
-        }
-    }
-    if (lane == 0) *tl = t;
-    __syncwarp();
+    return 2 * partial_blocks > blocks ? (int32_t)sched::MODE_CONTIG : (int32_t)sched::MODE_RR;
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -275,7 +241,6 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     __shared__ uint32_t s_tmem_base;
     __shared__ int32_t s_warp_sums[THREADS / 32];
     __shared__ SliceTable s_sl;
-    __shared__ sched::Tail s_tail;
     __shared__ int32_t s_blocks, s_partial;   // row blocks and partial ones (long tables)
 
     const int tid = threadIdx.x;
@@ -283,7 +248,6 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     const int lane = tid % 32;
 
     SegEntry* segs = reinterpret_cast<SegEntry*>(smem + geo.off_seg);
-    int32_t* inv = reinterpret_cast<int32_t*>(smem + geo.off_inv);
     PieceRec* recs = reinterpret_cast<PieceRec*>(smem + geo.off_q);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + geo.off_bar);
     const int SW = geo.stages_w, SXO = geo.stages_xo, SXR = geo.stages_xr;
@@ -431,13 +395,10 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
             total = long_table_total;
             mode = long_table_mode;
         }
-        if (mode == sched::MODE_BALANCED) build_tail(segs, nseg, total, geo.n_tiles, geo.halves, &s_tail, inv);
         if (lane == 0) {
             sched::Gen g;
             g.segs = segs;
             g.st = &s_sl;
-            g.inv = inv;
-            g.tl = &s_tail;
             g.nseg = nseg;
             g.n_tiles = geo.n_tiles;
             g.bn = BN;
@@ -876,8 +837,7 @@ constexpr int PIECE_FIXED_GROUPS = 0;
 
 // Shared-memory layout: an output ring of at least 4, else 3, 2, 1 whole
 // 128-row pieces, with the deepest B pipeline that leaves it room, after the
-// segment table (and, in the balanced mode, its bucket-sorted index) and the
-// piece queue.  In add mode the ring also holds the old output loaded ahead of
+// segment table and the piece queue.  In add mode the ring also holds the old output loaded ahead of
 // the epilogue, and the loads it can keep in flight set the pace: two B
 // stages, the rest for the ring (measured on one B200, us per call, 2 B
 // stages against the deepest that fits: rank-64 MLP 169.4 vs 178.3; QKV
@@ -892,7 +852,6 @@ inline bool layout_smem(Geometry& g, int32_t nseg, int32_t out_bytes, bool add, 
     const int32_t row_bytes = g.bn * out_bytes;            // one ring row across all chunks
     const int num_acc = TMEM_COLS / g.bn;
     const int32_t seg_bytes = round_up(nseg * (int32_t)sizeof(SegEntry), 16);
-    const int32_t inv_bytes = g.mode == MODE_AUTO && g.spread == sched::MODE_BALANCED ? round_up(nseg * 4, 16) : 0;
     const int32_t q_bytes = QS * (int32_t)sizeof(PieceRec);
     const int32_t budget = SMEM_OPTIN - SMEM_STATIC_RESERVE - 1024;   // 1024: base alignment slack
     for (int prefer_rows : {4 * BM, 3 * BM, 2 * BM, BM}) {
@@ -903,7 +862,7 @@ inline bool layout_smem(Geometry& g, int32_t nseg, int32_t out_bytes, bool add, 
             g.stages_xr = g.convert_x ? 1 : 0;
             const int n_bars = 2 * sw + 2 * g.stages_xo + 2 * g.stages_xr + 2 * num_acc + 2 * RING_PIECES + 2 * QS;
             const int32_t fixed = sw * g.w_bytes + g.stages_xo * g.xo_bytes + g.stages_xr * g.xr_bytes + seg_bytes +
-                                  inv_bytes + RING_PIECES * 4 + q_bytes + 8 * n_bars + 64;
+                                  RING_PIECES * 4 + q_bytes + 8 * n_bars + 64;
             if (fixed >= budget) continue;
             const int32_t rows = ((budget - fixed) / row_bytes) & ~(GROUP - 1);
             if (rows < prefer_rows) continue;
@@ -919,8 +878,6 @@ inline bool layout_smem(Geometry& g, int32_t nseg, int32_t out_bytes, bool add, 
             off += g.stages_xr * g.xr_bytes;
             g.off_seg = off;
             off += seg_bytes;
-            g.off_inv = off;
-            off += inv_bytes;
             g.off_ends = off;
             off += RING_PIECES * 4;
             g.off_q = round_up(off, 16);
@@ -998,8 +955,6 @@ inline bool make_plan_bn(const Problem* ps, int nsl, int sm_count, int bn, Plan*
     // must be rounded to the weights' dtype: that is done once per x block, so
     // a CTA then takes contiguous pieces and keeps a block across its n-tiles.
     g.mode = g.convert_x ? (int32_t)sched::MODE_CONTIG : MODE_AUTO;
-    g.spread = sched::MODE_RR;
-    g.halves = 2;
     g.wfix = (int32_t)wfix;
     // B tile: K in blocks of 64 columns, then at most one each of 32, 16, 8
     {

@@ -4,8 +4,8 @@ tests/sched_check.cpp compiles the scheduler header (csrc/tc_sched.cuh) for the
 host and enumerates the pieces of every CTA of a grid for random segment
 tables (empty, negative, over-long and unaligned segments, gaps, idle and
 out-of-range adapters), slice sets, tile widths and grid sizes, in both ways
-of handing out pieces, checking that every written element is covered
-exactly once and nothing else is.
+of handing out pieces (round-robin and contiguous), checking that every
+written element is covered exactly once and nothing else is.
 """
 import os
 import subprocess
@@ -21,6 +21,3 @@ def test_every_element_is_written_by_exactly_one_piece(tmp_path):
     r = subprocess.run([exe, "1500"], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "OK: 1500 cases" in r.stdout
-    # the balanced deal keeps the busiest CTA near the mean on a QKV-like batch
-    line = [l for l in r.stdout.splitlines() if l.startswith("qkv-like batch, halves 2")][0]
-    assert float(line.split()[-1]) < 1.02, line

@@ -46,6 +46,8 @@ import sgmv_inputs as gen  # noqa: E402
 METRIC = "sgmv_expand_slice achieved HBM GB/s (% of B200 roofline) and tokens/s per call"
 FALLBACK_HBM_GBS = 6650.0
 STEPS_PER_GRAPH = 100
+L2_BYTES = 126 << 20            # B200 L2
+MAX_COPIES = 8                  # most input copies a workload rotates through
 
 WORKLOAD_TEXT = {
     "qkv_prefill": "Llama-7B fused-QKV prefill: 16 seqs U[64,1024], rank 16, 32 adapters (10% idx -1), "
@@ -282,14 +284,20 @@ def make_multi_call(p, dev_tensors):
     return run
 
 
-def time_graph_region(step, steps, stream, torch):
+def graph_chunk(period):
+    """Steps per captured graph: at most STEPS_PER_GRAPH, a multiple of the
+    input rotation's period so that every replay continues the rotation."""
+    return max(period, STEPS_PER_GRAPH // period * period)
+
+
+def time_graph_region(step, steps, stream, torch, period=1):
     """Capture `steps` calls of step(stream_handle) as graphs of <= STEPS_PER_GRAPH
     steps, replay them once untimed, then time one replay of all of them with
     CUDA events on `stream`.  Returns milliseconds."""
     graphs = []
     remaining = steps
     while remaining > 0:
-        s = min(STEPS_PER_GRAPH, remaining)
+        s = min(graph_chunk(period), remaining)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             cs = torch.cuda.current_stream().cuda_stream
@@ -321,11 +329,43 @@ FLUSH_STEPS = 60             # steps of the flushed timing (median reported)
 EAGER_STEPS = 100            # steps of the eager (no graph) timing
 
 
+def footprint_bytes(p):
+    """Device bytes of a workload's buffers: x, the weights, the output and the metadata."""
+    return int(p.x.base.nbytes if p.x.base is not None else p.x.nbytes) + sum(int(c.w.nbytes) for c in p.calls) \
+        + int(p.y0.nbytes) + 3 * 8 * len(p.seq_start)
+
+
+def l2_copies(p):
+    """Copies of the workload's device buffers that the timed steps rotate through.
+
+    1 when one copy is larger than L2 (every step streams it from HBM anyway);
+    otherwise enough copies that the others, touched between two uses of one,
+    exceed L2, so that each step reads its inputs from HBM; at most MAX_COPIES.
+    Returns (copies, enough)."""
+    f = max(footprint_bytes(p), 1)
+    if f > L2_BYTES:
+        return 1, True
+    k = -(-L2_BYTES // f) + 1
+    return min(k, MAX_COPIES), k <= MAX_COPIES
+
+
+def l2_text(p):
+    k, enough = l2_copies(p)
+    mb = footprint_bytes(p) / 1e6
+    if k == 1:
+        return (f"no flush between steps: the step's buffers ({mb:.0f} MB) are larger than L2 and every step "
+                f"streams its output (a flushed median is reported beside it)")
+    if enough:
+        return (f"{k} copies of the inputs ({mb:.0f} MB each) used in turn: the {(k - 1) * mb:.0f} MB of the other "
+                f"copies touched between two uses of one exceed L2, so each step reads its inputs from HBM")
+    return (f"inputs of {mb:.2f} MB: {k} copies used in turn still fit in L2, so this is not an HBM-bound "
+            f"figure")
+
+
 def workload_config(p, name, world, step_fused=False):
     """The `config` object of a bench line: the workload, identical in both arms."""
     _, _, rows = step_accounting(p)
     ncalls = len(p.calls)
-    out_mb = p.y0.size * DT_SIZE[p.out_dt] / 1e6
     return {"workload": WORKLOAD_TEXT[name], "name": name,
             "batches": p.batches, "tokens_per_rank": p.total_tokens,
             "active_tokens_per_rank": rows // max(ncalls, 1), "rank": p.rank,
@@ -333,17 +373,19 @@ def workload_config(p, name, world, step_fused=False):
             "adapters": int(p.calls[0].w.shape[0]), "add_inputs": bool(p.add_inputs),
             "x_dtype": p.x_dt, "w_dtype": p.w_dt, "out_dtype": p.out_dt,
             "parallelism": f"replicas x{world} (independent batches, no collective)",
-            "l2": f"no flush between steps: every step streams the whole {out_mb:.0f} MB output, larger than L2 "
-                  f"(a flushed median is reported beside it)",
+            "l2": l2_text(p),
             "seed": p.seed,
             "step": ("all slices in one sgmv_expand_multi_slice call" if step_fused else
                      f"{ncalls} separate call(s)")}
 
 
 class Resident:
-    """A workload's inputs resident in HBM, with its C-ABI calls pre-marshalled."""
+    """A workload's inputs resident in HBM, with its C-ABI calls pre-marshalled.
 
-    def __init__(self, p, device):
+    With copies > 1 the device buffers exist that many times and step() uses
+    them in turn (see l2_copies); r.x, r.ws, r.y and r.meta are the first copy."""
+
+    def __init__(self, p, device, copies=1):
         import torch
         import segmented_gather_gemm_expand_b200 as sg
         self.p = p
@@ -367,6 +409,16 @@ class Resident:
             _, _, pref = sg.shrink_plan(x, ws[0], y, *meta, p.batches, p.max_seq_len, 1 << 34)
             self.workspace = torch.empty(max(pref, 16), dtype=torch.uint8, device=device)
         self.run, _ = make_calls(p, (x, ws, y, meta), None, None, workspace=self.workspace)
+        self.period = max(1, copies)
+        self.runs = [self.run]
+        self._copies = []
+        for _ in range(1, self.period):
+            cx, cws, cy = x.clone(), [w.clone() for w in ws], y.clone()
+            cmeta = [m.clone() for m in meta]
+            cwsp = torch.empty_like(self.workspace) if self.workspace is not None else None
+            self._copies.append((cx, cws, cy, cmeta, cwsp))
+            self.runs.append(make_calls(p, (cx, cws, cy, cmeta), None, None, workspace=cwsp)[0])
+        self.turn = 0
         self.ncalls = len(p.calls)
         self.shrink_splits = 0
         if p.op == "shrink":
@@ -385,6 +437,13 @@ class Resident:
         self.launches_per_call = 2 if (p.op == "shrink" and self.shrink_splits > 1) else 1
 
     def step(self, st):
+        """One step on the next copy of the buffers."""
+        run = self.runs[self.turn]
+        self.turn = (self.turn + 1) % self.period
+        for c in range(self.ncalls):
+            run(c, st)
+
+    def step_first_copy(self, st):
         for c in range(self.ncalls):
             self.run(c, st)
 
@@ -439,10 +498,11 @@ def secondary_entry(name, seed, steps, warmup, device, peak):
     import torch
     import segmented_gather_gemm_expand_b200 as sg
     p = gen.WORKLOADS[name](seed=seed)
-    r = Resident(p, device)
+    r = Resident(p, device, copies=l2_copies(p)[0])
     stream = torch.cuda.Stream(device)
     warm(r.step, warmup, stream, torch)
-    ms = time_graph_region(r.step, steps, stream, torch)
+    steps = -(-steps // r.period) * r.period
+    ms = time_graph_region(r.step, steps, stream, torch, r.period)
     assert sg.device_error(device) == 0, "a kernel reported a device-side error"
     b, f, rows = step_accounting(p)
     ncalls = r.ncalls
@@ -453,7 +513,7 @@ def secondary_entry(name, seed, steps, warmup, device, peak):
              "frac": call_bytes / (us_call * 1e-6) / 1e9 / peak,
              "tokens_per_s": p.total_tokens * steps / (ms * 1e-3),
              "tflops": f * steps / (ms * 1e-3) / 1e12, "bytes_per_call": call_bytes, "steps": steps,
-             "traffic": recorded_traffic(name, r.kernel_family)}
+             "traffic": recorded_traffic(name, r.kernel_family), "l2": l2_text(p)}
     del r
     torch.cuda.empty_cache()
     return entry
@@ -467,7 +527,7 @@ def bench_ours(args, rank, world, device):
     variants = {"auto": sg.VARIANT_AUTO, "simt": sg.VARIANT_SIMT, "tc": sg.VARIANT_TC}
     sg.set_variant(variants[args.variant])
     p = gen.WORKLOADS[args.workload](seed=args.seed + rank)
-    r = Resident(p, device)
+    r = Resident(p, device, copies=1 if args.step == "fused" else l2_copies(p)[0])
     ncalls = r.ncalls
     # One step: the slice calls one by one, or (--step fused) all slices in one
     # sgmv_expand_multi_slice call.
@@ -491,7 +551,7 @@ def bench_ours(args, rank, world, device):
     graphs = []
     remaining = K
     while remaining > 0:
-        s = min(STEPS_PER_GRAPH, remaining)
+        s = min(graph_chunk(r.period), remaining)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             cs = torch.cuda.current_stream().cuda_stream
@@ -597,7 +657,10 @@ def bench_ours(args, rank, world, device):
                     w.copy_(pw, non_blocking=True)
                 for m, pm in zip(r.meta, phmeta):
                     m.copy_(pm, non_blocking=True)
-                step_fn(stream.cuda_stream)
+                if fused_step:
+                    step_fn(stream.cuda_stream)
+                else:
+                    r.step_first_copy(stream.cuda_stream)
                 out_host.copy_(r.y, non_blocking=True)
             e1.record(stream)
         torch.cuda.synchronize()

@@ -118,6 +118,7 @@ int validate_call(const sgmv_tensor* x, const sgmv_tensor* w, const sgmv_tensor*
                   const sgmv_tensor* s, const sgmv_tensor* l, const sgmv_tensor* idx,
                   int64_t batches, int64_t max_seq_len, int64_t slice_offset, int64_t slice_size,
                   int add_inputs, Call* call) {
+    std::memset(call, 0, sizeof(Call));   // zeroed padding too: plans are cached by the bytes of the problem
     int rc;
     if ((rc = check_basic(x))) return rc;
     if ((rc = check_basic(w))) return rc;
@@ -379,7 +380,7 @@ int choose_shrink(const Call& c, const DeviceInfo& dev, int forced, const void* 
 
 int launch_shrink(const Call& c, const DeviceInfo& dev, int splits, float* ws, cudaStream_t stream) {
     shr::Plan pl;
-    if (!shr::make_plan(c.p, dev.sm_count, splits, tc::encode_fn(), &pl)) return SGMV_ERR_VARIANT;
+    if (!shr::cached_plan(c.p, dev.sm_count, splits, tc::encode_fn(), &pl)) return SGMV_ERR_VARIANT;
     switch (c.p.out_dt) {
         case SGMV_F32: return shr::launch_dt<SGMV_F32>(pl, c.p, ws, stream);
         case SGMV_BF16: return shr::launch_dt<SGMV_BF16>(pl, c.p, ws, stream);

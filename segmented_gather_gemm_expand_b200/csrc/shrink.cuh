@@ -6,10 +6,14 @@
 // It is the segmented product of the expand operation with the shapes turned
 // round: the reduction runs over the hidden size H (thousands) and the output
 // row is `rank` wide.  A work item is (segment, 128-row block, split of H).
-// Per 64-column chunk of H the producer warp TMA-loads the block's x rows (the
-// rows the segment owns, in 8..128-row boxes, 128-byte swizzle) and A[a]'s
-// rank x 64 tile; the MMA warp issues M=128, N=rank, K=16 tcgen05 MMAs into a
-// TMEM accumulator; the four epilogue warps read the sums back (one row per
+// H is cut into 64-column chunks; a pipeline stage holds up to four of them.
+// Per chunk the producer warp TMA-loads the block's x rows (the rows the
+// segment owns, in 8..128-row boxes, 128-byte swizzle) and A[a]'s rank x 64
+// tile, all chunks of a stage at once: with one chunk per stage the x stream
+// of the QKV shrink ran at about half the speed (a read-only TMA probe over a
+// 4096-wide bf16 matrix: 16.6 us with one 128 x 64 box per stage against 8.3
+// us with four neighbouring boxes per stage).  The MMA warp issues M=128,
+// N=rank, K=16 tcgen05 MMAs into a TMEM accumulator; the four epilogue warps read the sums back (one row per
 // thread) and either round them into out (one split) or store them as fp32
 // partial sums in the caller's workspace, which shrink_reduce_kernel adds up
 // in split order (deterministic) and rounds into out.
@@ -26,6 +30,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "plan_cache.cuh"
 #include "tc_ptx.cuh"
 
 namespace sgmv {
@@ -53,6 +58,7 @@ struct Geo {
     int32_t acc_stride;   // TMEM columns between the accumulators (R rounded up to 32)
     int32_t nchunks;      // ceil(H / CH)
     int32_t splits, cps;  // H splits per block; chunks per split
+    int32_t cpst;         // chunks per pipeline stage (1 to 4)
     int32_t stages, stage_bytes;
     int32_t off_seg, off_bar;
     int32_t tmem_cols;
@@ -197,20 +203,28 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
             for (int32_t id = blockIdx.x; ok && id < n_items; id += gridDim.x) {
                 decode_item(segs, nseg, g, full_blocks, id, it);
                 const int rows8 = (it.rows + 7) & ~7;
-                for (int32_t ch = it.ch0; ch < it.ch1; ++ch, ++q) {
+                for (int32_t ch = it.ch0; ch < it.ch1; ch += g.cpst, ++q) {
+                    const int nck = min(g.cpst, it.ch1 - ch);
                     const uint32_t s = q % S;
                     if (!mbar_wait(smem_u32(&empty[s]), ((q / S) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_PRODUCER)) {
                         ok = false;
                         break;
                     }
                     uint8_t* st = smem + s * g.stage_bytes;
-                    mbar_expect_tx(smem_u32(&full[s]), (uint32_t)(rows8 * 128 + g.R * 128));
-                    for (int r = 0; r < rows8;) {
-                        const int k = xbox_level(rows8 - r);
-                        tma_load_2d(smem_u32(st + r * 128), &xmaps.m[k], ch * CH, it.row0 + r, smem_u32(&full[s]), pol_x);
-                        r += 8 << k;
+                    uint8_t* sa = st + g.cpst * (BM * 128);
+                    mbar_expect_tx(smem_u32(&full[s]), (uint32_t)(nck * (rows8 * 128 + g.R * 128)));
+                    // the stage's chunks are requested together: neighbouring
+                    // 128-byte pieces of each x row are then in flight at once
+                    for (int j = 0; j < nck; ++j) {
+                        for (int r = 0; r < rows8;) {
+                            const int k = xbox_level(rows8 - r);
+                            tma_load_2d(smem_u32(st + j * (BM * 128) + r * 128), &xmaps.m[k], (ch + j) * CH,
+                                        it.row0 + r, smem_u32(&full[s]), pol_x);
+                            r += 8 << k;
+                        }
+                        tma_load_3d(smem_u32(sa + j * g.R * 128), &amap, (ch + j) * CH, 0, it.adapter,
+                                    smem_u32(&full[s]), pol_a);
                     }
-                    tma_load_3d(smem_u32(st + BM * 128), &amap, ch * CH, 0, it.adapter, smem_u32(&full[s]), pol_a);
                 }
             }
         }
@@ -225,7 +239,8 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
             if (!warp_wait(smem_u32(&acc_empty[acc]), ((n / NUM_ACC) & 1) ^ 1, abort_flag, DEVERR_TIMEOUT_MMA)) break;
             tc_fence_after();
             bool ok = true;
-            for (int32_t ch = it.ch0; ch < it.ch1; ++ch, ++q) {
+            for (int32_t ch = it.ch0; ch < it.ch1; ch += g.cpst, ++q) {
+                const int nck = min(g.cpst, it.ch1 - ch);
                 const uint32_t s = q % S;
                 if (!warp_wait(smem_u32(&full[s]), (q / S) & 1, abort_flag, DEVERR_TIMEOUT_MMA)) {
                     ok = false;
@@ -233,13 +248,17 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t xs = smem_u32(smem + s * g.stage_bytes);
-                    const uint32_t as = xs + BM * 128;
+                    const uint32_t st = smem_u32(smem + s * g.stage_bytes);
+                    for (int j = 0; j < nck; ++j) {
+                        const uint32_t xs = st + j * (BM * 128);
+                        const uint32_t as = st + g.cpst * (BM * 128) + j * g.R * 128;
 #pragma unroll
-                    for (int kk = 0; kk < CH / 16; ++kk) {
-                        const uint64_t ad = smem_desc(xs + kk * 32, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(as + kk * 32, 16, 1024, 2);
-                        tc_mma(tmem_base + acc * (uint32_t)g.acc_stride, ad, bd, idesc, (ch > it.ch0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < CH / 16; ++kk) {
+                            const uint64_t ad = smem_desc(xs + kk * 32, 16, 1024, 2);
+                            const uint64_t bd = smem_desc(as + kk * 32, 16, 1024, 2);
+                            tc_mma(tmem_base + acc * (uint32_t)g.acc_stride, ad, bd, idesc,
+                                   (ch > it.ch0 || j > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     tc_commit(smem_u32(&empty[s]));
                 }
@@ -304,19 +323,46 @@ shrink_kernel(const __grid_constant__ XMaps xmaps, const __grid_constant__ CUten
 }
 
 // Adds the splits' fp32 partial sums in split order and rounds each sum once
-// into out.  Grid: x = element chunks of a segment, y = segments (grid-stride).
+// into out.  A thread takes four neighbouring ranks of one row and issues the
+// loads of every split before it adds them (the sums are latency-bound: a few
+// MB that the main kernel has just written).  Grid: x = four-rank groups of a
+// segment, y = segments (grid-stride).  It lets the next kernel start its
+// prologue as soon as it runs.
+constexpr int MAX_SPLITS = 16;
+
 template <int OUT_DT>
 __global__ void __launch_bounds__(256) shrink_reduce_kernel(Problem p, const float* ws, int splits, int64_t t_lim) {
     grid_dependency_wait();   // the partial sums of the preceding shrink_kernel grid
-    const int64_t R = p.N;
+    grid_dependents_launch();
+    const int64_t R = p.N;    // a multiple of 16
+    const int64_t q = R / 4;
+    const int64_t split_stride = t_lim * R;
     for (int64_t b = blockIdx.y; b < p.batches; b += gridDim.y) {
         const Segment s = load_segment(p, b);
-        const int64_t n_el = s.rows * R;
-        for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_el; e += (int64_t)gridDim.x * blockDim.x) {
-            const int64_t row = s.row0 + e / R, k = e % R;
-            float acc = 0.f;
-            for (int sp = 0; sp < splits; ++sp) acc += ws[((int64_t)sp * t_lim + row) * R + k];
-            store_elem(p.out, OUT_DT, row * p.H + k, acc);
+        const int64_t n_vec = s.rows * q;
+        for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_vec; e += (int64_t)gridDim.x * blockDim.x) {
+            const int64_t row = s.row0 + e / q, k = (e % q) * 4;
+            const float4* src = reinterpret_cast<const float4*>(ws + row * R + k);
+            float4 v[MAX_SPLITS];
+#pragma unroll
+            for (int sp = 0; sp < MAX_SPLITS; ++sp)
+                if (sp < splits) v[sp] = src[sp * (split_stride / 4)];
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int sp = 0; sp < MAX_SPLITS; ++sp)
+                if (sp < splits) {
+                    acc.x += v[sp].x;
+                    acc.y += v[sp].y;
+                    acc.z += v[sp].z;
+                    acc.w += v[sp].w;
+                }
+            if (OUT_DT == SGMV_F32) {
+                *reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.H + k) = acc;
+            } else {
+                constexpr bool ob = OUT_DT == SGMV_BF16;
+                *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + row * p.H + k) =
+                    make_uint2(pack2(acc.x, acc.y, ob), pack2(acc.z, acc.w, ob));
+            }
         }
     }
 }
@@ -391,15 +437,23 @@ inline bool make_plan(const Problem& p, int sm_count, int splits, tc::EncodeTile
     g.nchunks = (int32_t)((p.K + CH - 1) / CH);
     g.cps = (g.nchunks + splits - 1) / splits;
     g.splits = (g.nchunks + g.cps - 1) / g.cps;                 // every split gets at least one chunk
+    if (g.splits > MAX_SPLITS) return false;
     g.t_lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
-    g.stage_bytes = BM * 128 + g.R * 128;                        // multiples of 1024: R % 16 == 0
-    for (g.stages = 8; g.stages >= 2; --g.stages) {
-        g.off_seg = g.stages * g.stage_bytes;
-        g.off_bar = (g.off_seg + (int)p.batches * (int)sizeof(SegRow) + 15) & ~15;
-        out->smem_bytes = g.off_bar + 8 * (2 * g.stages + 2 * NUM_ACC) + 1024;   // + base alignment slack
-        if (out->smem_bytes <= SMEM_LIMIT) break;
+    // A stage holds up to four chunks (x tiles, then the A tiles; every tile a
+    // multiple of 1024 bytes since R % 16 == 0): the widest stage of which at
+    // least two fit, then as many stages as fit, at most eight.
+    g.stages = 0;
+    for (g.cpst = g.cps < 4 ? g.cps : 4; g.cpst >= 1; g.cpst /= 2) {
+        g.stage_bytes = g.cpst * (BM * 128 + g.R * 128);
+        for (g.stages = 8; g.stages >= 2; --g.stages) {
+            g.off_seg = g.stages * g.stage_bytes;
+            g.off_bar = (g.off_seg + (int)p.batches * (int)sizeof(SegRow) + 15) & ~15;
+            out->smem_bytes = g.off_bar + 8 * (2 * g.stages + 2 * NUM_ACC) + 1024;   // + base alignment slack
+            if (out->smem_bytes <= SMEM_LIMIT) break;
+        }
+        if (g.stages >= 2) break;
     }
-    if (g.stages < 2) return false;
+    if (g.cpst < 1 || g.stages < 2) return false;
     g.acc_stride = (g.R + 31) / 32 * 32;
     int cols = 32;
     while (cols < NUM_ACC * g.acc_stride) cols *= 2;
@@ -433,6 +487,24 @@ inline bool make_plan(const Problem& p, int sm_count, int splits, tc::EncodeTile
     return true;
 }
 
+// Plans of recent calls, keyed by every field of the problem, the device, its
+// SM count and the split count.
+struct PlanKey {
+    Problem p;
+    int32_t device, sm_count, splits;
+};
+
+inline bool cached_plan(const Problem& p, int sm_count, int splits, tc::EncodeTiledFn enc, Plan* out) {
+    static PlanCache<PlanKey, Plan> cache;
+    PlanKey key;
+    std::memset(&key, 0, sizeof(key));
+    std::memcpy(&key.p, &p, sizeof(Problem));
+    key.sm_count = sm_count;
+    key.splits = splits;
+    if (cudaGetDevice(&key.device) != cudaSuccess) return false;
+    return cache.get(key, out, [&](Plan* pl) { return make_plan(p, sm_count, splits, enc, pl); });
+}
+
 template <int OUT_DT>
 int launch_dt(const Plan& pl, const Problem& p, float* ws, cudaStream_t stream) {
     auto kern = shrink_kernel<OUT_DT>;
@@ -454,7 +526,7 @@ int launch_dt(const Plan& pl, const Problem& p, float* ws, cudaStream_t stream) 
     if (cudaLaunchKernelEx(&cfg, kern, pl.xm, pl.am, p, pl.geo, ws) != cudaSuccess) return SGMV_ERR_LAUNCH;
     if (pl.geo.splits > 1) {
         const int64_t rows_guess = (pl.geo.t_lim + p.batches - 1) / (p.batches > 0 ? p.batches : 1);
-        int64_t gx = (rows_guess * p.N + 255) / 256;
+        int64_t gx = (rows_guess * (p.N / 4) + 255) / 256;
         if (gx < 1) gx = 1;
         if (gx > 1024) gx = 1024;
         cudaLaunchConfig_t rc = {};

@@ -47,9 +47,11 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
+#include "plan_cache.cuh"
 #include "tc_ptx.cuh"
 #include "tc_sched.cuh"
 
@@ -1110,11 +1112,32 @@ int launch_instance(const Plan& pl, const Problem& p, cudaStream_t stream) {
     return SGMV_OK;
 }
 
+// Plans of recent calls, keyed by every field of the call's slices (pointers,
+// dtypes, shapes, strides, metadata, slice offsets and widths, add mode), the
+// device, its SM count and the tile width asked for.
+struct PlanKey {
+    Problem ps[MAX_SLICES];
+    int32_t nsl, device, sm_count, force_bn;
+};
+
+inline bool cached_plan(const Problem* ps, int nsl, int sm_count, int force_bn, Plan* out) {
+    static PlanCache<PlanKey, Plan> cache;
+    if (nsl < 1 || nsl > MAX_SLICES) return false;
+    PlanKey key;
+    std::memset(&key, 0, sizeof(key));
+    for (int i = 0; i < nsl; ++i) std::memcpy(&key.ps[i], &ps[i], sizeof(Problem));
+    key.nsl = nsl;
+    key.sm_count = sm_count;
+    key.force_bn = force_bn;
+    if (cudaGetDevice(&key.device) != cudaSuccess) return false;
+    return cache.get(key, out, [&](Plan* pl) { return make_plan(ps, nsl, sm_count, pl, force_bn); });
+}
+
 }  // namespace tc
 
 bool tc_supports(const Problem* ps, int nsl, int sm_count, int force_bn) {
     tc::Plan pl;
-    return tc::make_plan(ps, nsl, sm_count, &pl, force_bn);
+    return tc::cached_plan(ps, nsl, sm_count, force_bn, &pl);
 }
 
 template <int BN>
@@ -1134,7 +1157,7 @@ int launch_bn(const tc::Plan& pl, const Problem& p, cudaStream_t stream) {
 
 int launch_tc(const Problem* ps, int nsl, int sm_count, cudaStream_t stream, int force_bn) {
     tc::Plan pl;
-    if (!tc::make_plan(ps, nsl, sm_count, &pl, force_bn)) return SGMV_ERR_VARIANT;
+    if (!tc::cached_plan(ps, nsl, sm_count, force_bn, &pl)) return SGMV_ERR_VARIANT;
     const Problem& p = ps[0];
     return pl.geo.bn == 256 ? launch_bn<256>(pl, p, stream) : launch_bn<128>(pl, p, stream);
 }

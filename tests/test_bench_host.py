@@ -49,6 +49,32 @@ def test_step_sums_its_calls():
     assert bench.step_accounting(p) == tuple(sum(v[i] for v in per_call) for i in range(3))
 
 
+@pytest.mark.parametrize("name", sorted(gen.WORKLOADS))
+def test_timed_steps_read_their_inputs_from_hbm(name):
+    """Workloads whose buffers fit in L2 rotate through copies of them: between two uses of a copy the
+    other copies touched exceed L2 (tiny, at a few kilobytes, cannot and says so)."""
+    p = gen.WORKLOADS[name]()
+    k, enough = bench.l2_copies(p)
+    f = bench.footprint_bytes(p)
+    assert 1 <= k <= bench.MAX_COPIES
+    if k == 1:
+        assert f > bench.L2_BYTES
+    elif enough:
+        assert (k - 1) * f > bench.L2_BYTES and (k - 2) * f <= bench.L2_BYTES
+    else:
+        assert name == "tiny" and "not an HBM-bound figure" in bench.l2_text(p)
+    if name in ("qkv_shrink", "decode_bgmv"):
+        assert k > 1 and enough
+    if name in ("qkv_prefill", "mlp_mixed", "long_single", "decode_mix"):
+        assert k == 1
+
+
+def test_graph_chunks_keep_the_rotation():
+    for period in range(1, bench.MAX_COPIES + 1):
+        c = bench.graph_chunk(period)
+        assert c % period == 0 and period <= c <= max(bench.STEPS_PER_GRAPH, period)
+
+
 def test_every_kernel_family_hashes_existing_sources():
     csrc = os.path.join(bench.ROOT, "segmented_gather_gemm_expand_b200", "csrc")
     for family, files in bench.KERNEL_SOURCES.items():

@@ -80,6 +80,12 @@ constexpr int MAX_WBLK = 4;           // B tile K blocks (64/32/16/8 columns)
 constexpr int MAX_SLICES = sched::MAX_SLICES;   // slices of one output updated by one launch
 constexpr int RING_PIECES = 32;       // pieces that may hold ring space at once
 constexpr int QS = 64;                // piece records in the queue
+// Records a short table's scheduler prepares before the dependency wait.  The
+// table's load and scan there are what pays; each held record delays the
+// start if the wait ends first.  QKV prefill, us per call by held records
+// 0/1/2/4/16: 29.2, 28.8, 28.8, 30.4, 35.6 (30.3 with the table built after
+// the wait); the single-tenant batch 48.9, 49.2, 49.6, 50.9, 55.7 (48.5).
+constexpr int SPEC_RECORDS = 1;
 // an accumulator slot, a ring barrier slot and a queue slot always serve the same epilogue group
 static_assert(RING_PIECES % EPI_GROUPS == 0 && QS % EPI_GROUPS == 0, "slot ownership");
 constexpr int32_t MODE_AUTO = -1;     // Geometry::mode: decided on the device from the segment table
@@ -156,6 +162,29 @@ struct PieceRec {
 
 // log2 of the lanes between repeats of a block's rows in the staged x operand:
 // the rows rounded up to 32, 64 or 128.
+// load_segment read through L2 (ld.global.cg), same guards.  The scheduler of
+// a short table reads the metadata once before the preceding grid may have
+// finished and once after; the second read must not hit a stale L1 line.
+__device__ __forceinline__ int64_t load_meta_l2(const MetaVec& m, int64_t i) {
+    if (m.dtype == META_IOTA) return i;
+    if (m.dtype == META_ONE) return 1;
+    if (m.dtype == SGMV_I64) return __ldcg(reinterpret_cast<const long long*>(m.ptr) + i * m.stride);
+    return (int64_t)__ldcg(reinterpret_cast<const int*>(m.ptr) + i * m.stride);
+}
+
+__device__ __forceinline__ Segment load_segment_l2(const Problem& p, int64_t b) {
+    Segment s;
+    s.row0 = load_meta_l2(p.start, b);
+    const int64_t L = load_meta_l2(p.len, b);
+    s.adapter = load_meta_l2(p.idx, b);
+    const int64_t lim = p.out_rows < p.x_rows ? p.out_rows : p.x_rows;
+    int64_t end = s.row0 + L;
+    if (end > lim) end = lim;
+    const bool ok = s.adapter >= 0 && s.adapter < p.lora_num && s.row0 >= 0 && L > 0 && end > s.row0;
+    s.rows = ok ? end - s.row0 : 0;
+    return s;
+}
+
 __host__ __device__ __forceinline__ int32_t x_period_log(int32_t rows) { return rows <= 32 ? 5 : rows <= 64 ? 6 : BM_LOG; }
 
 // Place a piece of rows8 rows in a ring of R rows: returns the ring row where it
@@ -337,8 +366,11 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
     __syncthreads();
     tc_fence_after();
 
-    // Everything below may read memory written by the preceding kernel.
-    grid_dependency_wait();
+    // Everything below may read memory written by the preceding kernel.  (The
+    // scheduler warp of a short segment table waits by itself, after it has
+    // prepared its first records from a speculative read of the metadata.)
+    const bool sched_spec = p.batches <= WARP_TABLE_MAX;
+    if (!(warp == SCHED_WARP && sched_spec)) grid_dependency_wait();
     // The next kernel may be scheduled now: its CTAs take SMs as ours leave, and
     // it waits for this grid to finish before it reads anything.
     grid_dependents_launch();
@@ -372,97 +404,148 @@ tc_expand_slice_kernel(const __grid_constant__ WMaps wmaps, const __grid_constan
 
     if (warp == SCHED_WARP) {
         // ------------------------------------------------------------ scheduler
-        int32_t total, mode;
-        if (nseg <= WARP_TABLE_MAX) {
-            // a short table: one segment per lane, a warp scan, no block barrier
-            SegEntry e{0, 0, 0, 0};
-            if (lane < nseg) {
-                const Segment s = load_segment(p, lane);
-                e = SegEntry{(int32_t)s.row0, (int32_t)s.rows, (int32_t)s.adapter, 0};
-            }
-            mode = choose_mode(geo, (int32_t)__reduce_add_sync(0xffffffffu, (e.rows % BM) != 0 ? 1u : 0u),
-                               (int32_t)__reduce_add_sync(0xffffffffu, (uint32_t)((e.rows + BM - 1) / BM)));
-            const int32_t units = lane < nseg ? seg_units(geo, mode, e.rows) : 0;
-            int32_t v = units;
+        // A short table is read and scanned, and its first SPEC_RECORDS record(s)
+        // generated into the queue without being published, while the
+        // preceding grid may still run.  After the dependency wait the warp
+        // reads the metadata again: if it is unchanged the held records are
+        // published at once and generation goes on; if not, everything is
+        // redone from the new table (pass 1).  Long tables are built by the
+        // whole block after the wait and go straight to pass 1.
+        bool retry = false;
+#pragma unroll 1
+        for (int pass = sched_spec ? 0 : 1; pass < 2; ++pass) {
+            int spec_bit = pass == 0;
+            asm volatile("" : "+r"(spec_bit));   // one copy of the code for both passes
+            const bool spec = spec_bit != 0;
+            int32_t total, mode;
+            SegEntry mine{0, 0, 0, 0};             // this lane's segment (short tables)
+            if (nseg <= WARP_TABLE_MAX) {
+                if (!spec) grid_dependency_wait();   // (again after a failed speculation: returns at once)
+                // a short table: one segment per lane, a warp scan, no block barrier
+                SegEntry e{0, 0, 0, 0};
+                if (lane < nseg) {
+                    const Segment sg = load_segment_l2(p, lane);
+                    e = SegEntry{(int32_t)sg.row0, (int32_t)sg.rows, (int32_t)sg.adapter, 0};
+                }
+                mine = e;
+                mode = choose_mode(geo, (int32_t)__reduce_add_sync(0xffffffffu, (e.rows % BM) != 0 ? 1u : 0u),
+                                   (int32_t)__reduce_add_sync(0xffffffffu, (uint32_t)((e.rows + BM - 1) / BM)));
+                const int32_t units = lane < nseg ? seg_units(geo, mode, e.rows) : 0;
+                int32_t v = units;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += t;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += t;
+                }
+                e.prefix = v - units;
+                if (lane < nseg) segs[lane] = e;
+                total = __shfl_sync(0xffffffffu, v, 31);
+                __syncwarp();
+            } else {
+                total = long_table_total;
+                mode = long_table_mode;
             }
-            e.prefix = v - units;
-            if (lane < nseg) segs[lane] = e;
-            total = __shfl_sync(0xffffffffu, v, 31);
-            __syncwarp();
-        } else {
-            total = long_table_total;
-            mode = long_table_mode;
-        }
-        if (lane == 0) {
-            sched::Gen g;
-            g.segs = segs;
-            g.st = &s_sl;
-            g.nseg = nseg;
-            g.n_tiles = geo.n_tiles;
-            g.bn = BN;
-            g.mode = mode;
-            g.init((int32_t)blockIdx.x, (int32_t)gridDim.x, total, geo.wmin, geo.wfix);
             constexpr int CC_LOG = OUT_BYTES == 4 ? 5 : 6;
+            sched::Gen g;
             Piece cur, nxt, prev;
-            bool have = g.next(cur), ok = true;
+            bool have = false, ok = true;
             int32_t t = 0, head = 0, prev_seg = -1, prev_rb = -1;
-            while (have && ok) {
-                const bool have_n = g.next(nxt);
-                PieceRec r;
-                r.adapter = cur.adapter;
-                r.blk_row0 = cur.blk_row0;
-                r.rows = cur.rows;
-                r.n0 = cur.n0;
-                r.col0 = cur.col0;
-                r.ncols = cur.ncols;
-                r.slice = cur.slice;
-                r.flags = 0;
-                if (cur.seg != prev_seg || cur.rb != prev_rb) r.flags |= REC_NEW_X;
-                if (!have_n || nxt.seg != cur.seg || nxt.rb != cur.rb) r.flags |= REC_LAST_X;
-                if (t == 0 || cur.adapter != prev.adapter || cur.slice != prev.slice || cur.n0 != prev.n0)
-                    r.flags |= REC_NEW_W;
-                if (!have_n || nxt.adapter != cur.adapter || nxt.slice != cur.slice || nxt.n0 != cur.n0)
-                    r.flags |= REC_LAST_W;
-                // A short piece (rows in 1 or 2 quadrants) is computed in every span
-                // of 32 or 64 lanes: the x block is staged with its rows repeated
-                // (x_period), so each TMEM quadrant holds a copy of the sums, and the
-                // epilogue warps of the copies split the piece's column chunks.  Where
-                // the piece has fewer chunks than copies, its rows instead take turns
-                // in the lanes of a wider span (the pieces of one epilogue group,
-                // every EPI_GROUPS-th, cycle through them).
-                const int32_t span_log = x_period_log(cur.rows);
-                const int32_t nch = (cur.ncols + (1 << CC_LOG) - 1) >> CC_LOG;
-                const int32_t maxrep_log = BM_LOG - span_log;
-                r.rep_log = min(maxrep_log, nch >= 4 ? 2 : nch >= 2 ? 1 : 0);
-                const int32_t turns_mask = (1 << (maxrep_log - r.rep_log)) - 1;
-                r.shift = ((t / EPI_GROUPS) & turns_mask) << span_log;
-                r.pos = ring_place(head, (cur.rows + GROUP - 1) & ~(GROUP - 1), R);
-                r.head_end = head;
-                const int slot = t % QS;
-                if (!mbar_wait(smem_u32(&q_empty[slot]), ((t / QS) & 1) ^ 1, abort_flag, DEVERR_SCHEDULE)) {
-                    ok = false;
+            if (lane == 0) {
+                g.segs = segs;
+                g.st = &s_sl;
+                g.nseg = nseg;
+                g.n_tiles = geo.n_tiles;
+                g.bn = BN;
+                g.mode = mode;
+                g.init((int32_t)blockIdx.x, (int32_t)gridDim.x, total, geo.wmin, geo.wfix);
+                have = g.next(cur);
+            }
+            // phase 0 (speculative): up to SPEC_RECORDS records, held; phase 1: the rest
+#pragma unroll 1
+            for (int phase = spec ? 0 : 1; phase < 2; ++phase) {
+                const bool hold = phase == 0;
+                const int32_t stop = hold ? SPEC_RECORDS : 0x7fffffff;
+                if (lane == 0) {
+                    while (have && ok && t < stop) {
+                        const bool have_n = g.next(nxt);
+                        PieceRec r;
+                        r.adapter = cur.adapter;
+                        r.blk_row0 = cur.blk_row0;
+                        r.rows = cur.rows;
+                        r.n0 = cur.n0;
+                        r.col0 = cur.col0;
+                        r.ncols = cur.ncols;
+                        r.slice = cur.slice;
+                        r.flags = 0;
+                        if (cur.seg != prev_seg || cur.rb != prev_rb) r.flags |= REC_NEW_X;
+                        if (!have_n || nxt.seg != cur.seg || nxt.rb != cur.rb) r.flags |= REC_LAST_X;
+                        if (t == 0 || cur.adapter != prev.adapter || cur.slice != prev.slice || cur.n0 != prev.n0)
+                            r.flags |= REC_NEW_W;
+                        if (!have_n || nxt.adapter != cur.adapter || nxt.slice != cur.slice || nxt.n0 != cur.n0)
+                            r.flags |= REC_LAST_W;
+                        // A short piece (rows in 1 or 2 quadrants) is computed in every span
+                        // of 32 or 64 lanes: the x block is staged with its rows repeated
+                        // (x_period), so each TMEM quadrant holds a copy of the sums, and the
+                        // epilogue warps of the copies split the piece's column chunks.  Where
+                        // the piece has fewer chunks than copies, its rows instead take turns
+                        // in the lanes of a wider span (the pieces of one epilogue group,
+                        // every EPI_GROUPS-th, cycle through them).
+                        const int32_t span_log = x_period_log(cur.rows);
+                        const int32_t nch = (cur.ncols + (1 << CC_LOG) - 1) >> CC_LOG;
+                        const int32_t maxrep_log = BM_LOG - span_log;
+                        r.rep_log = min(maxrep_log, nch >= 4 ? 2 : nch >= 2 ? 1 : 0);
+                        const int32_t turns_mask = (1 << (maxrep_log - r.rep_log)) - 1;
+                        r.shift = ((t / EPI_GROUPS) & turns_mask) << span_log;
+                        r.pos = ring_place(head, (cur.rows + GROUP - 1) & ~(GROUP - 1), R);
+                        r.head_end = head;
+                        const int slot = t % QS;
+                        // (held records fit the queue: SPEC_RECORDS <= QS, so this wait
+                        // passes at once in phase 0)
+                        if (!mbar_wait(smem_u32(&q_empty[slot]), ((t / QS) & 1) ^ 1, abort_flag, DEVERR_SCHEDULE)) {
+                            ok = false;
+                            break;
+                        }
+                        recs[slot] = r;
+                        if (!hold) mbar_arrive(smem_u32(&q_full[slot]));
+                        prev_seg = cur.seg;
+                        prev_rb = cur.rb;
+                        prev = cur;
+                        cur = nxt;
+                        have = have_n;
+                        ++t;
+                    }
+                }
+                __syncwarp();
+                if (!hold) break;
+                // the speculation is confirmed if every lane's segment reads the same now
+                grid_dependency_wait();
+                bool same = true;
+                if (lane < nseg) {
+                    const Segment sg = load_segment_l2(p, lane);
+                    same = sg.row0 == mine.row0 && sg.rows == mine.rows && sg.adapter == mine.adapter;
+                }
+                if (!__all_sync(0xffffffffu, same)) {
+                    retry = true;
                     break;
                 }
-                recs[slot] = r;
-                mbar_arrive(smem_u32(&q_full[slot]));
-                prev_seg = cur.seg;
-                prev_rb = cur.rb;
-                prev = cur;
-                cur = nxt;
-                have = have_n;
-                ++t;
+                if (lane == 0)   // publish the held records
+                    for (int32_t i = 0; i < t; ++i) mbar_arrive(smem_u32(&q_full[i % QS]));
+                __syncwarp();
+            }
+            if (retry && pass == 0) {
+                retry = false;
+                continue;   // pass 1: the table again, after the wait, nothing held
             }
             // one end record for each epilogue group (the other roles stop at the first)
-            for (int e = 0; ok && e < EPI_GROUPS; ++e, ++t) {
-                const int slot = t % QS;
-                if (!mbar_wait(smem_u32(&q_empty[slot]), ((t / QS) & 1) ^ 1, abort_flag, DEVERR_SCHEDULE)) break;
-                recs[slot].flags = REC_END;
-                mbar_arrive(smem_u32(&q_full[slot]));
+            if (lane == 0) {
+                for (int e = 0; ok && e < EPI_GROUPS; ++e, ++t) {
+                    const int slot = t % QS;
+                    if (!mbar_wait(smem_u32(&q_empty[slot]), ((t / QS) & 1) ^ 1, abort_flag, DEVERR_SCHEDULE)) break;
+                    recs[slot].flags = REC_END;
+                    mbar_arrive(smem_u32(&q_full[slot]));
+                }
             }
+            break;
         }
         __syncwarp();
     } else if (warp == 0) {

@@ -735,8 +735,11 @@ def bench_ours(args, rank, world, device):
                      "kernel": f"{ {'bgmv': 'bgmv_expand_slice', 'shrink': 'sgmv_shrink'}.get(p.op, 'sgmv_expand_slice') } "
                                f"({r.variant}{', %d H splits + reduction' % r.shrink_splits if r.shrink_splits > 1 else ''})",
                      "launch_ms_avg": avg_launch_ms, "bytes_per_launch": call_bytes,
+                     "launch_sm_cycles": (avg_launch_ms * 1e-3 * clocks["sm_mhz"] * 1e6
+                                          if clocks and clocks.get("sm_mhz") else None),
                      "launches_timed": K * calls_per_step,
-                     "launch_ms_note": "timed region / calls (back-to-back calls, gaps included; a split shrink "
+                     "launch_ms_note": "timed region / calls (back-to-back calls, gaps included; launch_sm_cycles = "
+                                       "that time x the median SM clock sampled during the region; a split shrink "
                                        "call is its main kernel plus the reduction)"},
         "gpu_launches": K * launches_per_step,
         "clocks": clocks,

@@ -85,6 +85,16 @@ def test_bgmv_batches_smaller_than_rows(variant):
     run_bgmv(p, BGMV_VARIANTS[variant], batches=23)
 
 
+@pytest.mark.parametrize("K,pad", [(32, 8), (64, 16), (16, 0), (8, 0)])
+def test_bgmv_dense_and_padded_b_rows(K, pad):
+    """Dense and padded B rows (row stride K or K + pad) both take the decode kernel; slices of 1, 255, 256
+    and 257 columns cover a CTA's 256-column tile whole, partly and with one column over."""
+    for N in (1, 255, 256, 257):
+        p = bgmv_problem(K + N + pad, B=37, K=K, N=N, H=N + 40, off=24, A=4, w_row_pad=pad,
+                         idx=[(i * 3) % 6 - 1 for i in range(37)])
+        assert run_bgmv(p, sg.VARIANT_AUTO) == sg.VARIANT_DECODE
+
+
 def test_bgmv_strided_x_takes_the_decode_kernel():
     p = bgmv_problem(5, B=20, K=24, N=96, H=192, off=96, A=3, x_col_pad=3)
     assert run_bgmv(p, sg.VARIANT_AUTO) == sg.VARIANT_DECODE

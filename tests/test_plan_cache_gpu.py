@@ -95,3 +95,24 @@ def test_shrink_same_buffers_other_workspace():
         assert sg.device_error() == 0
         _, count = compare_every_element(y.cpu().numpy(), ref, p, [(rows, 0, 16)])
         assert count == int(rows.sum()) * 16
+
+
+def test_metadata_written_on_the_device_just_before_the_call():
+    """The scheduler of a short segment table reads the metadata before the preceding kernel may have
+    finished and checks it again afterwards; here a device copy rewrites the metadata right before each
+    call (same stream, no synchronisation), alternating between two batches of different lengths."""
+    lengths_a = [300, 50, 700, 130]
+    lengths_b = [700, 130, 50, 300]
+    pa = gen.custom(7, lengths=lengths_a, **SHAPE)
+    pb = gen.custom(7, lengths=lengths_b, idx=[1, 3, -1, 0], **SHAPE)
+    pb.x = pa.x
+    pb.calls[0] = pa.calls[0]
+    dp = DeviceProblem(pa)
+    meta = {"a": meta_tensors(pa), "b": meta_tensors(pb)}
+    for name, p in (("b", pb), ("a", pa), ("b", pb)):
+        dp.y = to_torch(p.y0, p.out_dt)
+        for mine, new in zip((dp.start, dp.len, dp.idx), meta[name]):
+            mine.copy_(new, non_blocking=True)
+        dp.p = p
+        dp.run()
+        check(dp, p)

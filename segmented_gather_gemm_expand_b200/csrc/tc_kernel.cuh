@@ -160,8 +160,6 @@ struct PieceRec {
                           // REC_NEW_W / REC_LAST_W: the same for its B tile (adapter, slice, first column)
 };
 
-// log2 of the lanes between repeats of a block's rows in the staged x operand:
-// the rows rounded up to 32, 64 or 128.
 // load_segment read through L2 (ld.global.cg), same guards.  The scheduler of
 // a short table reads the metadata once before the preceding grid may have
 // finished and once after; the second read must not hit a stale L1 line.
@@ -185,6 +183,8 @@ __device__ __forceinline__ Segment load_segment_l2(const Problem& p, int64_t b) 
     return s;
 }
 
+// log2 of the lanes between repeats of a block's rows in the staged x operand:
+// the rows rounded up to 32, 64 or 128.
 __host__ __device__ __forceinline__ int32_t x_period_log(int32_t rows) { return rows <= 32 ? 5 : rows <= 64 ? 6 : BM_LOG; }
 
 // Place a piece of rows8 rows in a ring of R rows: returns the ring row where it
